@@ -1,0 +1,330 @@
+// C ABI of the Domino draft-block library (declared in include/domino.h).
+//
+// Host side only: argument validation, workspace carve-up and the launch
+// sequence.  Every step of the path runs in the kernels of this library.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "../../include/domino.h"
+#include "common.cuh"
+#include "domino_internal.h"
+
+using domino::Control;
+
+namespace {
+
+std::atomic<uint64_t> g_budget_ns{2000000000ull};
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+struct Layout {
+  size_t ctl, base, S, u, best, end;                       // device workspace
+  size_t h_hidden, h_anchor, h_forced, h_target, h_draft, h_tau, h_end;  // host-variant staging
+};
+
+bool weights_ok(const domino_weights* w) {
+  if (!w) return false;
+  if (w->dtype != DOMINO_BF16 && w->dtype != DOMINO_F32) return false;
+  if (w->vocab < 1 || w->d_model < 8 || w->embed_dim < 8 || w->gru_hidden < 8 || w->rank < 8) return false;
+  if (w->d_model % 8 || w->embed_dim % 8 || w->gru_hidden % 8 || w->rank % 8) return false;
+  return true;
+}
+
+bool weight_ptrs_ok(const domino_weights* w, bool need_lm, bool need_loop) {
+  if (need_lm && (!w->w_lm || !aligned16(w->w_lm))) return false;
+  if (need_loop) {
+    const void* req[] = {w->embed, w->w_ih, w->w_hh, w->w1, w->w2};
+    for (const void* p : req)
+      if (!p || !aligned16(p)) return false;
+    if (w->b_ih && !aligned16(w->b_ih)) return false;
+    if (w->b_hh && !aligned16(w->b_hh)) return false;
+  }
+  return true;
+}
+
+Layout layout_of(const domino_weights* w, int B, int K) {
+  Layout L{};
+  const size_t wb = w->dtype == DOMINO_BF16 ? 2 : 4;
+  size_t o = 0;
+  L.ctl = o; o += align_up(sizeof(Control));
+  L.base = o; o += align_up(static_cast<size_t>(B) * K * w->vocab * 4);
+  L.S = o; o += align_up(2ull * 8 * w->gru_hidden * 4);
+  L.u = o; o += align_up(8ull * w->rank * 4);
+  L.best = o; o += align_up(static_cast<size_t>(K) * 8 * 8);
+  L.end = o;
+  L.h_hidden = o; o += align_up(static_cast<size_t>(B) * K * w->d_model * wb);
+  L.h_anchor = o; o += align_up(static_cast<size_t>(B) * 4);
+  L.h_forced = o; o += align_up(static_cast<size_t>(B) * K * 4);
+  L.h_target = o; o += align_up(static_cast<size_t>(B) * K * 4);
+  L.h_draft = o; o += align_up(static_cast<size_t>(B) * K * 4);
+  L.h_tau = o; o += align_up(static_cast<size_t>(B) * 4);
+  L.h_end = o;
+  return L;
+}
+
+domino_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return DOMINO_OK;
+  (void)cudaGetLastError();
+  if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorLaunchOutOfResources) return DOMINO_ERR_LAUNCH;
+  return DOMINO_ERR_CUDA;
+}
+
+domino_status check_workspace(void* ws, size_t bytes, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || bytes < need) return DOMINO_ERR_WORKSPACE;
+  return DOMINO_OK;
+}
+
+domino_status run_lm_head(const domino_weights* w, const void* hidden, int B, int K, float* base, Control* ctl,
+                          cudaStream_t st) {
+  const int M = B * K;
+  cudaError_t e;
+  if (w->dtype == DOMINO_BF16) {
+    const int sms = num_sms();
+    if (sms <= 0) return DOMINO_ERR_CUDA;
+    e = domino::launch_lm_head_tc(w->w_lm, hidden, base, w->vocab, M, w->d_model, ctl, g_budget_ns.load(), sms, st);
+  } else {
+    e = domino::launch_lm_head_f32(static_cast<const float*>(w->w_lm), static_cast<const float*>(hidden), base,
+                                   w->vocab, M, w->d_model, st);
+  }
+  return from_cuda(e);
+}
+
+domino_status run_loop(const domino_weights* w, const void* hidden, const float* base, const int32_t* anchor, int B,
+                       int K, int mode, float temperature, uint64_t seed, const int32_t* forced,
+                       const int32_t* target, int32_t* draft, float* logits, int32_t* tau, char* ws, const Layout& L,
+                       cudaStream_t st) {
+  const int sms = num_sms();
+  if (sms <= 0) return DOMINO_ERR_CUDA;
+  const size_t wb = w->dtype == DOMINO_BF16 ? 2 : 4;
+  const int NB = domino::loop_group_size(B);
+  domino::LoopArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.embed = w->embed;
+  a.w_ih = w->w_ih;
+  a.w_hh = w->w_hh;
+  a.b_ih = w->b_ih;
+  a.b_hh = w->b_hh;
+  a.w1 = w->w1;
+  a.w2 = w->w2;
+  a.ctl = reinterpret_cast<Control*>(ws + L.ctl);
+  a.S_glob = reinterpret_cast<float*>(ws + L.S);
+  a.u_glob = reinterpret_cast<float*>(ws + L.u);
+  a.best = reinterpret_cast<unsigned long long*>(ws + L.best);
+  a.seed = seed;
+  a.budget_ns = g_budget_ns.load();
+  a.temperature = temperature;
+  a.V = w->vocab;
+  a.d = w->d_model;
+  a.E = w->embed_dim;
+  a.H = w->gru_hidden;
+  a.r = w->rank;
+  a.K = K;
+  a.mode = mode;
+  a.wbytes = static_cast<int>(wb);
+  const size_t smem = domino::loop_plan(a, NB, sms, 227 * 1024);
+  if (smem == 0) return DOMINO_ERR_UNSUPPORTED;
+  for (int g0 = 0; g0 < B; g0 += NB) {
+    const int nb = B - g0 < NB ? B - g0 : NB;
+    domino::LoopArgs g = a;
+    g.b0 = g0;
+    g.nb = nb;
+    g.hidden = static_cast<const char*>(hidden) + static_cast<size_t>(g0) * K * w->d_model * wb;
+    g.base = base + static_cast<size_t>(g0) * K * w->vocab;
+    g.anchor = anchor + g0;
+    g.forced = forced ? forced + static_cast<size_t>(g0) * K : nullptr;
+    g.target = target ? target + static_cast<size_t>(g0) * K : nullptr;
+    g.draft = draft + static_cast<size_t>(g0) * K;
+    g.logits = logits ? logits + static_cast<size_t>(g0) * K * w->vocab : nullptr;
+    g.tau = tau ? tau + g0 : nullptr;
+    const domino_status s = from_cuda(domino::launch_correct_loop(g, NB, sms, smem, st));
+    if (s != DOMINO_OK) return s;
+  }
+  return DOMINO_OK;
+}
+
+domino_status validate_block(const domino_weights* w, const void* hidden, const int32_t* anchor, int B, int K,
+                             int mode, float temperature, const int32_t* forced, const int32_t* target,
+                             const void* draft_out, const void* logits_out, const void* tau_out) {
+  if (!weights_ok(w)) return DOMINO_ERR_INVALID_ARG;
+  if (B < 1 || K < 1 || K > 32) return DOMINO_ERR_INVALID_ARG;
+  if (mode != DOMINO_GREEDY && mode != DOMINO_GUMBEL) return DOMINO_ERR_INVALID_ARG;
+  if (mode == DOMINO_GUMBEL && !(temperature > 0.f && std::isfinite(temperature))) return DOMINO_ERR_INVALID_ARG;
+  if (!hidden || !aligned16(hidden) || !anchor || !aligned16(anchor)) return DOMINO_ERR_INVALID_ARG;
+  if (!draft_out || !aligned16(draft_out)) return DOMINO_ERR_INVALID_ARG;
+  if (forced && !aligned16(forced)) return DOMINO_ERR_INVALID_ARG;
+  if (target && (!aligned16(target) || !tau_out || !aligned16(tau_out))) return DOMINO_ERR_INVALID_ARG;
+  if (logits_out && !aligned16(logits_out)) return DOMINO_ERR_INVALID_ARG;
+  const int rmax = w->dtype == DOMINO_BF16 ? 256 : 128;
+  if (w->rank > rmax) return DOMINO_ERR_UNSUPPORTED;
+  return DOMINO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t domino_workspace_bytes(const domino_weights* w, int32_t B, int32_t K) {
+  if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return 0;
+  return layout_of(w, B, K).end;
+}
+
+size_t domino_workspace_bytes_host(const domino_weights* w, int32_t B, int32_t K) {
+  if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return 0;
+  return layout_of(w, B, K).h_end;
+}
+
+domino_status domino_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < sizeof(Control))
+    return DOMINO_ERR_WORKSPACE;
+  return from_cuda(cudaMemsetAsync(workspace, 0, sizeof(Control), static_cast<cudaStream_t>(stream)));
+}
+
+domino_status domino_lm_head(const domino_weights* w, const void* hidden, int32_t B, int32_t K, float* base_out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!weights_ok(w) || !weight_ptrs_ok(w, true, false)) return DOMINO_ERR_INVALID_ARG;
+  if (B < 1 || K < 1 || K > 32 || !hidden || !aligned16(hidden) || !base_out || !aligned16(base_out))
+    return DOMINO_ERR_INVALID_ARG;
+  const domino_status ws = check_workspace(workspace, workspace_bytes, sizeof(Control));
+  if (ws != DOMINO_OK) return ws;
+  return run_lm_head(w, hidden, B, K, base_out, static_cast<Control*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+domino_status domino_correct_loop(const domino_weights* w, const void* hidden, const float* base,
+                                  const int32_t* anchor, int32_t B, int32_t K, int32_t mode, float temperature,
+                                  uint64_t seed, const int32_t* forced, const int32_t* target, int32_t* draft_out,
+                                  float* logits_out, int32_t* tau_out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  domino_status s = validate_block(w, hidden, anchor, B, K, mode, temperature, forced, target, draft_out,
+                                   logits_out, tau_out);
+  if (s != DOMINO_OK) return s;
+  if (!weight_ptrs_ok(w, false, true) || !base || !aligned16(base)) return DOMINO_ERR_INVALID_ARG;
+  const Layout L = layout_of(w, B, K);
+  s = check_workspace(workspace, workspace_bytes, L.end);
+  if (s != DOMINO_OK) return s;
+  return run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out,
+                  tau_out, static_cast<char*>(workspace), L, static_cast<cudaStream_t>(stream));
+}
+
+domino_status domino_draft_block(const domino_weights* w, const void* hidden, const int32_t* anchor, int32_t B,
+                                 int32_t K, int32_t mode, float temperature, uint64_t seed, const int32_t* forced,
+                                 const int32_t* target, int32_t* draft_out, float* logits_out, int32_t* tau_out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  domino_status s = validate_block(w, hidden, anchor, B, K, mode, temperature, forced, target, draft_out,
+                                   logits_out, tau_out);
+  if (s != DOMINO_OK) return s;
+  if (!weight_ptrs_ok(w, true, true)) return DOMINO_ERR_INVALID_ARG;
+  const Layout L = layout_of(w, B, K);
+  s = check_workspace(workspace, workspace_bytes, L.end);
+  if (s != DOMINO_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* base = reinterpret_cast<float*>(ws + L.base);
+  s = run_lm_head(w, hidden, B, K, base, reinterpret_cast<Control*>(ws + L.ctl), st);
+  if (s != DOMINO_OK) return s;
+  return run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out,
+                  tau_out, ws, L, st);
+}
+
+domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K, int32_t* tau_out,
+                            void* stream) {
+  if (!draft || !target || !tau_out || B < 1 || K < 1 || K > 32) return DOMINO_ERR_INVALID_ARG;
+  if (!aligned16(draft) || !aligned16(target) || !aligned16(tau_out)) return DOMINO_ERR_INVALID_ARG;
+  return from_cuda(domino::launch_verify(draft, target, B, K, tau_out, static_cast<cudaStream_t>(stream)));
+}
+
+domino_status domino_draft_block_host(const domino_weights* w, const void* hidden_host, const int32_t* anchor_host,
+                                      int32_t B, int32_t K, int32_t mode, float temperature, uint64_t seed,
+                                      const int32_t* forced_host, const int32_t* target_host,
+                                      int32_t* draft_out_host, int32_t* tau_out_host, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return DOMINO_ERR_INVALID_ARG;
+  if (!hidden_host || !anchor_host || !draft_out_host || (target_host && !tau_out_host)) return DOMINO_ERR_INVALID_ARG;
+  const Layout L = layout_of(w, B, K);
+  domino_status s = check_workspace(workspace, workspace_bytes, L.h_end);
+  if (s != DOMINO_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t wb = w->dtype == DOMINO_BF16 ? 2 : 4;
+  const size_t tok = static_cast<size_t>(B) * K * 4;
+  cudaError_t e = cudaMemcpyAsync(ws + L.h_hidden, hidden_host, static_cast<size_t>(B) * K * w->d_model * wb,
+                                  cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.h_anchor, anchor_host, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && forced_host) e = cudaMemcpyAsync(ws + L.h_forced, forced_host, tok, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && target_host) e = cudaMemcpyAsync(ws + L.h_target, target_host, tok, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  int32_t* d_draft = reinterpret_cast<int32_t*>(ws + L.h_draft);
+  int32_t* d_tau = reinterpret_cast<int32_t*>(ws + L.h_tau);
+  s = domino_draft_block(w, ws + L.h_hidden, reinterpret_cast<const int32_t*>(ws + L.h_anchor), B, K, mode,
+                         temperature, seed, forced_host ? reinterpret_cast<const int32_t*>(ws + L.h_forced) : nullptr,
+                         target_host ? reinterpret_cast<const int32_t*>(ws + L.h_target) : nullptr, d_draft, nullptr,
+                         target_host ? d_tau : nullptr, workspace, L.end, stream);
+  if (s != DOMINO_OK) return s;
+  e = cudaMemcpyAsync(draft_out_host, d_draft, tok, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess && target_host)
+    e = cudaMemcpyAsync(tau_out_host, d_tau, static_cast<size_t>(B) * 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return from_cuda(e);
+}
+
+domino_status domino_poll(void* workspace, void* stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return DOMINO_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t err = 0;
+  cudaError_t e = cudaMemcpyAsync(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (err == 0) return DOMINO_OK;
+  e = cudaMemsetAsync(workspace, 0, sizeof(Control), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (err & domino::ERRBIT_TIMEOUT) return DOMINO_ERR_TIMEOUT;
+  return DOMINO_ERR_BAD_TOKEN;
+}
+
+void domino_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns ? ns : 1); }
+
+domino_status domino_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t budget_ns, void* stream) {
+  const domino_status s = check_workspace(workspace, workspace_bytes, sizeof(Control));
+  if (s != DOMINO_OK) return s;
+  const int sms = num_sms();
+  if (sms <= 0) return DOMINO_ERR_CUDA;
+  domino::LoopArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.ctl = static_cast<Control*>(workspace);
+  a.budget_ns = budget_ns;
+  a.selftest = 1;
+  a.wbytes = 2;
+  a.nslot = 0;
+  const domino_status ls =
+      from_cuda(domino::launch_correct_loop(a, 1, sms, 1024, static_cast<cudaStream_t>(stream)));
+  if (ls != DOMINO_OK) return ls;
+  return domino_poll(workspace, stream);
+}
+
+const char* domino_status_str(domino_status s) {
+  switch (s) {
+    case DOMINO_OK: return "DOMINO_OK";
+    case DOMINO_ERR_INVALID_ARG: return "DOMINO_ERR_INVALID_ARG";
+    case DOMINO_ERR_UNSUPPORTED: return "DOMINO_ERR_UNSUPPORTED";
+    case DOMINO_ERR_LAUNCH: return "DOMINO_ERR_LAUNCH";
+    case DOMINO_ERR_CUDA: return "DOMINO_ERR_CUDA";
+    case DOMINO_ERR_TIMEOUT: return "DOMINO_ERR_TIMEOUT";
+    case DOMINO_ERR_BAD_TOKEN: return "DOMINO_ERR_BAD_TOKEN";
+    case DOMINO_ERR_WORKSPACE: return "DOMINO_ERR_WORKSPACE";
+  }
+  return "DOMINO_ERR_UNKNOWN";
+}
+
+}  // extern "C"

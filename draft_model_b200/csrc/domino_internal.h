@@ -1,0 +1,74 @@
+// Internal declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace domino {
+
+struct Control;
+
+// Bytes per slot of the correction loop's weight ring.
+constexpr uint32_t kLoopSlotBytes = 16384;
+
+// Launch arguments of the persistent correction-loop kernel (one request group).
+struct LoopArgs {
+  // weights
+  const void* embed;
+  const void* w_ih;
+  const void* w_hh;
+  const float* b_ih;
+  const float* b_hh;
+  const void* w1;
+  const void* w2;
+  // inputs (already offset to the group's first request)
+  const void* hidden;   // [nb, K, d]
+  const float* base;    // [nb, K, V]
+  const int32_t* anchor;
+  const int32_t* forced;  // or null
+  const int32_t* target;  // or null
+  // outputs (offset to the group)
+  int32_t* draft;
+  float* logits;        // or null
+  int32_t* tau;         // or null
+  // scratch
+  Control* ctl;
+  float* S_glob;                 // [2][NB][H]
+  float* u_glob;                 // [NB][r]
+  unsigned long long* best;      // [K][NB]
+  uint64_t seed;
+  uint64_t budget_ns;
+  float temperature;
+  int32_t V, d, E, H, r, K;
+  int32_t b0;       // global index of the group's first request (Philox counter)
+  int32_t nb;       // requests in this group (<= NB)
+  int32_t mode;     // 0 greedy, 1 Gumbel
+  int32_t wbytes;   // 2 (bf16) or 4 (f32)
+  int32_t selftest; // 1: run only the unreachable-barrier self-test
+  // segment plan
+  int32_t segE3, nsegE3, segH3, nsegH3, segH1, nsegH1;
+  int32_t max_part;
+  int32_t nslot;
+  // shared-memory carve-up (byte offsets)
+  uint32_t off_bars, off_S, off_x, off_u, off_part, off_hp, off_tok, off_wbest, off_flags;
+};
+
+// Fills the segment plan and shared-memory offsets; returns the dynamic shared
+// memory size, or 0 if the shapes do not fit.
+size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap);
+int loop_group_size(int B);
+int loop_threads();
+cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaStream_t stream);
+
+// LM head (stage 1).
+cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd,
+                              Control* ctl, uint64_t budget_ns, int num_sms, cudaStream_t stream);
+cudaError_t launch_lm_head_f32(const float* w_lm, const float* hidden, float* out, int V, int M, int Kd,
+                               cudaStream_t stream);
+
+// Verification (stage 3).
+cudaError_t launch_verify(const int32_t* draft, const int32_t* target, int B, int K, int32_t* tau,
+                          cudaStream_t stream);
+
+}  // namespace domino

@@ -1,0 +1,326 @@
+// Stage 1 of the Domino draft block on the tcgen05 tensor cores (sm_100a):
+// base logits L^base[m, v] = sum_k W_lm[v, k] h[m, k] for every block position m
+// (m = b*K + i), computed once per block (Domino study notes, gsyq.cn, §二.1(1);
+// yhxrc.cn article, §三 第一个阶段).
+//
+// Swap-AB formulation: the UMMA "A" operand is a 128-row tile of W_lm (vocabulary
+// on the M side, so V = 151936 = 1187 x 128 tiles exactly) and "B" is a tile of
+// the hidden states (BN = 16..256 block positions on the N side).  The fp32
+// accumulator lives in tensor memory: TMEM lane = vocabulary row, column = block
+// position, so the epilogue's tcgen05.ld hands every thread one vocabulary row
+// and a warp stores 32 consecutive floats of one output row (coalesced).
+//
+// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: 2-D tiled loads (128B swizzle) of A and B into a
+//               STAGES-deep shared-memory ring (no multicast);
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//               (tcgen05.mma.cta_group::1.kind::f16, K = 16 per instruction);
+//   warps 2..5  epilogue: tcgen05.ld 32x32b from a double-buffered accumulator,
+//               fp32 stores to HBM while the next tile accumulates.
+// Every mbarrier wait is bounded; on expiry the kernel flags DOMINO_ERR_TIMEOUT,
+// drains its copies and MMAs, frees TMEM and returns.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "domino_internal.h"
+
+namespace domino {
+namespace {
+
+constexpr int BM = 128;        // vocabulary rows per tile (UMMA M)
+constexpr int BK = 64;         // bf16 elements per k-block (one 128-byte swizzle atom row)
+constexpr int NTH = 192;
+constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;  // 16 KB
+
+struct TcArgs {
+  float* out;
+  Control* ctl;
+  uint64_t budget_ns;
+  int V, M, Kd;
+  int BN;            // block positions per tile (multiple of 16, <= 256)
+  int stages;
+  int tmem_cols;     // power of two >= 2*BN
+  int num_vt, num_mt, num_kb;
+};
+
+// ---- tcgen05 / TMA primitives (inline PTX) ----
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(tm), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(tm) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, int ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, int ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
+// atoms 1024 bytes apart (stride byte offset), sm100 descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);          // start address
+  d |= static_cast<uint64_t>(1u) << 16;                        // leading byte offset (unused for SW128 K-major)
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;                // stride byte offset
+  d |= static_cast<uint64_t>(1u) << 46;                        // descriptor version
+  d |= static_cast<uint64_t>(2u) << 61;                        // SWIZZLE_128B
+  return d;
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major, M=128, N=BN.
+__device__ __forceinline__ uint32_t idesc_bf16_f32(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(NTH, 1)
+    lm_head_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment of every stage (the swizzle atom)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t b_stage_bytes = static_cast<uint32_t>(a.BN) * BK * 2;
+  const uint32_t stage_bytes = A_STAGE_BYTES + b_stage_bytes;
+  uint8_t* ctrl = smem + static_cast<size_t>(a.stages) * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + a.stages;
+  uint64_t* tfull = empty + a.stages;   // [2]
+  uint64_t* tempty = tfull + 2;         // [2]
+  uint64_t* mma_done = tempty + 2;      // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = a.num_vt * a.num_mt;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, a.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto bounded_wait = [&](uint64_t* bar, uint32_t par) -> bool {
+    if (*abort_flag) return false;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, par)) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > a.budget_ns) {
+        raise_error(a.ctl, ERRBIT_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  };
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int it = 0;  // global k-block counter
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int vt = t / a.num_mt, mt = t % a.num_mt;
+        for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+          const int s = it % a.stages;
+          if (it >= a.stages && !bounded_wait(&empty[s], ((it / a.stages) - 1) & 1)) { ok = false; break; }
+          uint8_t* sa = smem + static_cast<size_t>(s) * stage_bytes;
+          uint8_t* sb = sa + A_STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], stage_bytes);
+          tma_load_2d(sa, &tmA, kb * BK, vt * BM, &full[s]);
+          tma_load_2d(sb, &tmB, kb * BK, mt * a.BN, &full[s]);
+        }
+      }
+      // drain copies that were issued but may still be in flight
+      for (int j = max(0, it - a.stages); j < it; ++j) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[j % a.stages], (j / a.stages) & 1)) {
+          if (globaltimer_ns() - t0 > a.budget_ns) { raise_error(a.ctl, ERRBIT_TIMEOUT); break; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(a.BN);
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        if (local >= 2 && !bounded_wait(&tempty[acc], ((local >> 1) - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
+        for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+          const int s = it % a.stages;
+          if (!bounded_wait(&full[s], (it / a.stages) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+          const uint32_t sb = sa + A_STAGE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            tc_mma_bf16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);   // frees the stage once these MMAs have read it
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      // every MMA issued by this thread must finish before TMEM is released
+      tc_commit(mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(mma_done, 0)) {
+        if (globaltimer_ns() - t0 > a.budget_ns) { raise_error(a.ctl, ERRBIT_TIMEOUT); break; }
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4
+    const int q = warp & 3;
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      bool ok = true;
+      if (lane == 0) ok = bounded_wait(&tfull[acc], (local >> 1) & 1);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const int vt = t / a.num_mt, mt = t % a.num_mt;
+      const int v = vt * BM + q * 32 + lane;
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      for (int c0 = 0; c0 < a.BN; c0 += 16) {
+        float vals[16];
+        tmem_ld16(trow + c0, vals);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int m = mt * a.BN + c0 + c;
+          if (v < a.V && m < a.M) a.out[static_cast<size_t>(m) * a.V + v] = vals[c];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, a.tmem_cols);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* tm, const void* ptr, int rows, int cols, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd, Control* ctl,
+                              uint64_t budget_ns, int num_sms, cudaStream_t stream) {
+  TcArgs a;
+  a.out = out;
+  a.ctl = ctl;
+  a.budget_ns = budget_ns;
+  a.V = V;
+  a.M = M;
+  a.Kd = Kd;
+  int bn = (M + 15) / 16 * 16;
+  a.BN = bn > 256 ? 256 : bn;
+  int cols = 32;
+  while (cols < 2 * a.BN) cols <<= 1;
+  a.tmem_cols = cols;
+  a.num_vt = (V + BM - 1) / BM;
+  a.num_mt = (M + a.BN - 1) / a.BN;
+  a.num_kb = (Kd + BK - 1) / BK;
+  const uint32_t stage_bytes = A_STAGE_BYTES + static_cast<uint32_t>(a.BN) * BK * 2;
+  const size_t budget = 220 * 1024;
+  int stages = static_cast<int>((budget - 2048) / stage_bytes);
+  if (stages > 12) stages = 12;
+  if (stages < 2) return cudaErrorInvalidValue;
+  a.stages = stages;
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes + 1024 /*align*/ + 256 /*barriers*/;
+
+  CUtensorMap tmA, tmB;
+  if (!make_tmap(&tmA, w_lm, V, Kd, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tmB, hidden, M, Kd, a.BN)) return cudaErrorInvalidValue;
+
+  cudaError_t e = cudaFuncSetAttribute(lm_head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int ntiles = a.num_vt * a.num_mt;
+  const int grid = ntiles < num_sms ? ntiles : num_sms;
+  lm_head_tc_kernel<<<grid, NTH, smem, stream>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace domino

@@ -171,12 +171,15 @@ class Result:
 def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
                 mode: str = "greedy", temperature: float = 1.0, seed: int = 0,
                 forced: np.ndarray | None = None, target: np.ndarray | None = None,
-                want_logits: bool = True, base: np.ndarray | None = None) -> Result:
+                want_logits: bool = True, base: np.ndarray | None = None,
+                request_ids: np.ndarray | None = None) -> Result:
     """Run one draft block for every request.
 
     hidden: storage-form [B, K, d]; anchor: [B] int.  ``forced`` [B, K] feeds
     forced[b, i] to the GRU after position i instead of the pick (the last
     column is never fed).  ``base`` may pass precomputed fp64 base logits.
+    ``request_ids`` [B] names each row's request index in the Gumbel stream
+    (default 0..B-1), so a sample of a larger batch draws the same noise.
     """
     if mode not in ("greedy", "gumbel"):
         raise ValueError(mode)
@@ -194,6 +197,7 @@ def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
     gap = np.zeros((B, K)) if forced is not None else None
     logits = np.zeros((B, K, V)) if want_logits else None
 
+    rid = np.arange(B) if request_ids is None else np.asarray(request_ids, dtype=np.int64)
     s = np.zeros((B, H))
     prev = np.asarray(anchor, dtype=np.int64).copy()
     for p in range(K):                      # block position i = p + 1
@@ -207,7 +211,7 @@ def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
         if mode == "greedy":
             score = L
         else:
-            g = np.stack([gumbel_noise(seed, b, p + 1, V) for b in range(B)])
+            g = np.stack([gumbel_noise(seed, int(rid[b]), p + 1, V) for b in range(B)])
             score = L / temperature + g
         pick = np.argmax(score, axis=1)      # first index among equal maxima
         tokens[:, p] = pick

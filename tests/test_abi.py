@@ -1,0 +1,108 @@
+"""C-ABI checks that need no GPU: the library builds and loads, it exports every
+entry point include/domino.h declares, and host-side validation rejects bad
+arguments synchronously (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import draft_model_b200 as dm
+from draft_model_b200 import build as dbuild
+from draft_model_b200._binding import _CWeights
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "domino.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dbuild.build()
+    return dm.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"DOMINO_API\s+[\w\s\*]+?\b(domino_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("domino_draft_block", "domino_lm_head", "domino_correct_loop", "domino_verify", "domino_poll",
+                 "domino_status_str", "domino_workspace_bytes"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(dm.library_path())
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} declared in domino.h but not exported"
+
+
+def test_status_strings(lib):
+    for code, name in dm.STATUS.items():
+        assert dm.domino_status_str(code) == name
+    assert dm.domino_status_str(99) == "DOMINO_ERR_UNKNOWN"
+
+
+def _cw(V=151936, d=4096, E=4096, H=1024, r=256, dtype=0, ptr=0x10000):
+    p = ctypes.c_void_p(ptr)
+    return _CWeights(V, d, E, H, r, dtype, p, p, p, p, None, None, p, p)
+
+
+def test_workspace_bytes(lib):
+    w = _cw()
+    n = lib.domino_workspace_bytes(ctypes.byref(w), 1, 16)
+    # control block + base logits (B*K*V fp32) + GRU state + u + argmax keys, 256-aligned pieces
+    assert n >= 16 * 151936 * 4 + 256
+    assert n % 256 == 0
+    assert lib.domino_workspace_bytes(ctypes.byref(w), 2, 16) > n
+    assert lib.domino_workspace_bytes_host(ctypes.byref(w), 1, 16) > n
+    assert lib.domino_workspace_bytes(ctypes.byref(w), 0, 16) == 0
+    assert lib.domino_workspace_bytes(ctypes.byref(w), 1, 33) == 0
+    bad = _cw(d=4095)
+    assert lib.domino_workspace_bytes(ctypes.byref(bad), 1, 16) == 0
+
+
+def _block(lib, w, *, B=1, K=16, mode=0, T=1.0, hidden=0x20000, anchor=0x30000, draft=0x40000, target=None,
+           tau=None, ws=0x100000, wsn=1 << 40):
+    return lib.domino_draft_block(ctypes.byref(w), hidden, anchor, B, K, mode, T, 0, None, target, draft, None, tau,
+                                  ws, wsn, None)
+
+
+def test_validation_is_synchronous_and_host_side(lib):
+    w = _cw()
+    INVALID, UNSUP, WS = 1, 2, 7
+    assert _block(lib, w, B=0) == INVALID
+    assert _block(lib, w, K=0) == INVALID
+    assert _block(lib, w, K=33) == INVALID
+    assert _block(lib, w, mode=2) == INVALID
+    assert _block(lib, w, mode=1, T=0.0) == INVALID
+    assert _block(lib, w, mode=1, T=float("nan")) == INVALID
+    assert _block(lib, w, hidden=None) == INVALID
+    assert _block(lib, w, hidden=0x20001) == INVALID          # misaligned
+    assert _block(lib, w, draft=None) == INVALID
+    assert _block(lib, w, target=0x50000, tau=None) == INVALID  # tau needed with a target
+    assert _block(lib, _cw(r=264)) == UNSUP                     # rank above the bf16 limit
+    assert _block(lib, _cw(dtype=1, r=136)) == UNSUP            # rank above the f32 limit
+    assert _block(lib, _cw(dtype=3)) == INVALID
+    assert _block(lib, w, ws=None) == WS
+    assert _block(lib, w, ws=0x100010) == WS                    # workspace not 256-aligned
+    assert _block(lib, w, wsn=1024) == WS                       # workspace too small
+    nullw = _cw(ptr=0)
+    assert _block(lib, nullw) == INVALID
+
+
+def test_verify_and_init_validation(lib):
+    assert lib.domino_verify(0x1000, 0x2000, 1, 33, 0x3000, None) == 1
+    assert lib.domino_verify(None, 0x2000, 1, 4, 0x3000, None) == 1
+    assert lib.domino_verify(0x1000, 0x2000, 0, 4, 0x3000, None) == 1
+    assert lib.domino_workspace_init(0x1001, 4096, None) == 7
+    assert lib.domino_workspace_init(0x1000, 16, None) == 7
+
+
+def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
+    from draft_model_b200 import _binding
+    monkeypatch.setattr(_binding, "_lib", None)
+    monkeypatch.setattr(_binding, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _binding.load_library()
