@@ -51,6 +51,8 @@ def load_library() -> ctypes.CDLL:
         "domino_workspace_bytes_host": (SZ, [W, I32, I32]),
         "domino_workspace_init": (I32, [P, SZ, P]),
         "domino_draft_block": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
+        "domino_draft_block_events": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P,
+                                             ctypes.POINTER(ctypes.c_void_p)]),
         "domino_lm_head": (I32, [W, P, I32, I32, P, P, SZ, P]),
         "domino_correct_loop": (I32, [W, P, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
         "domino_verify": (I32, [P, P, I32, I32, P, P]),
@@ -150,6 +152,19 @@ def domino_draft_block(w: DominoWeights, hidden, anchor, *, mode=0, temperature=
     _check(load_library().domino_draft_block(w.ref, _ptr(hidden), _ptr(anchor), B, K, mode, temperature, seed,
                                              _ptr(forced), _ptr(target), _ptr(draft_out), _ptr(logits_out),
                                              _ptr(tau_out), wp, wn, _stream(stream)), "domino_draft_block")
+
+
+def domino_draft_block_events(w: DominoWeights, hidden, anchor, *, mode=0, temperature=1.0, seed=0, forced=None,
+                              target=None, draft_out, logits_out=None, tau_out=None, workspace, stream=None,
+                              events) -> None:
+    """domino_draft_block recording three torch.cuda.Event objects around its stages."""
+    B, K = draft_out.shape
+    wp, wn = _ws(workspace)
+    arr = (ctypes.c_void_p * 3)(*[None if e is None else e.cuda_event for e in events])
+    _check(load_library().domino_draft_block_events(w.ref, _ptr(hidden), _ptr(anchor), B, K, mode, temperature, seed,
+                                                    _ptr(forced), _ptr(target), _ptr(draft_out), _ptr(logits_out),
+                                                    _ptr(tau_out), wp, wn, _stream(stream), arr),
+           "domino_draft_block_events")
 
 
 def domino_lm_head(w: DominoWeights, hidden, base_out, *, workspace, stream=None) -> None:

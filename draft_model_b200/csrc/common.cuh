@@ -19,8 +19,8 @@ constexpr uint32_t ERRBIT_BAD_TOKEN = 2u;
 // Workspace control block (first 256 bytes of every workspace).
 struct Control {
   uint32_t err;          // ERRBIT_* accumulated by device code
-  uint32_t bar_count;    // grid barrier: arrivals in the current episode
-  uint32_t bar_gen;      // grid barrier: completed episodes
+  uint32_t bar_count;    // grid barrier: arrivals during the current launch
+  uint32_t bar_gen;      // CTAs that have left the current launch
   uint32_t pad0;
   uint64_t pad[30];
 };
@@ -53,29 +53,42 @@ __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
 }
 
 // Grid-wide barrier for a co-resident (cooperatively launched) grid, executed by
-// ONE thread per CTA (the caller brackets it with a CTA barrier).  Sense via a
-// generation counter: the last arriver resets the arrival count and bumps the
-// generation, so the control block is clean after every episode.  Returns false
-// if the wait ran out of budget (the error bit is raised).
-__device__ __forceinline__ bool grid_barrier_one_thread(Control* ctl, uint32_t nblocks, uint64_t budget_ns) {
-  const uint32_t gen = ld_acquire_u32(&ctl->bar_gen);
-  const uint32_t arrived = atom_add_release_u32(&ctl->bar_count, 1u) + 1u;
-  if (arrived == nblocks) {
-    st_relaxed_u32(&ctl->bar_count, 0u);
-    atom_add_release_u32(&ctl->bar_gen, 1u);
-    return true;
-  }
-  const uint64_t t0 = globaltimer_ns();
+// ONE thread per CTA (the caller brackets it with a CTA barrier).  The arrival
+// counter only grows during a launch: barrier number k (0-based) completes when
+// it reaches G*(k+1).  Arrival is a fire-and-forget release reduction; the wait
+// polls with relaxed loads and ends with an acquire fence.  The last CTA to
+// leave the kernel resets the counter (grid_exit), so every launch starts at 0.
+// Returns false if the wait ran out of budget (the error bit is raised).
+__device__ __forceinline__ bool grid_barrier_one_thread(Control* ctl, uint32_t target, uint64_t budget_ns) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&ctl->bar_count) : "memory");
   uint32_t spins = 0;
-  while (ld_acquire_u32(&ctl->bar_gen) == gen) {
-    if ((++spins & 63u) == 0u) {
-      if (globaltimer_ns() - t0 > budget_ns) {
+  uint64_t t0 = 0;
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&ctl->bar_count) : "memory");
+    if (static_cast<int32_t>(v - target) >= 0) break;
+    if ((++spins & 31u) == 0u) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > budget_ns) {
         raise_error(ctl, ERRBIT_TIMEOUT);
         return false;
       }
     }
   }
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
   return true;
+}
+
+// Called once per CTA (one thread) after its last barrier: the last CTA out
+// resets the barrier counter for the next launch on this workspace.
+__device__ __forceinline__ void grid_exit(Control* ctl, uint32_t nblocks) {
+  const uint32_t n = atom_add_release_u32(&ctl->bar_gen, 1u) + 1u;
+  if (n == nblocks) {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    st_relaxed_u32(&ctl->bar_count, 0u);
+    st_relaxed_u32(&ctl->bar_gen, 0u);
+  }
 }
 
 // ---------------------------------------------------------------- shared-memory mbarriers
@@ -127,6 +140,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+// Bulk prefetch of a global range into L2 (no shared-memory destination).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+// 4-byte asynchronous global -> shared copy (LDGSTS) and its group fences.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

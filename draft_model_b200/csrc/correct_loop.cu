@@ -16,16 +16,17 @@
 //   * a contiguous vocabulary range [v0, v1) of W2 (balanced so every CTA streams
 //     about the same number of weight bytes per step).
 // A producer warp streams exactly those weight bytes, step after step, through a
-// shared-memory ring with 1-D bulk copies (TMA engine, no tensor map).  The
-// weights never depend on data, so the producer runs ahead across the grid
-// barriers and HBM stays busy while consumers wait for data dependencies.
-// Four consumer warps compute from the ring; item n is always handled by warp
-// n % 4 and lands in slot n % NSLOT (NSLOT a multiple of 4), so a slot is only
-// ever waited on by the warp that consumed its previous occupant.
+// shared-memory ring with 1-D bulk copies (TMA engine, no tensor map), and
+// issues bulk L2 prefetches a fixed distance ahead of the ring.  The weights
+// never depend on data, so HBM keeps streaming while consumers wait on grid
+// barriers.  Four consumer warps compute from the ring; item n is always handled
+// by warp n % 4 and lands in slot n % NSLOT (NSLOT a multiple of 4), so a slot is
+// only ever waited on by the warp that consumed its previous occupant.
 // Per step three bounded grid barriers: after the GRU (S_i complete), after the
 // bottleneck (u complete), after the vocabulary pass (argmax keys merged with a
 // 64-bit atomicMax).  W1 [h_i ; S] is split as W1_h h_i + W1_s S; the W1_h h_i
-// terms of the CTA's own rows are computed once for all positions up front.
+// terms come precomputed from stage 1.  The CTA's slice of the base logits for
+// step i is copied into shared memory with cp.async while the GRU runs.
 // Delta L and L_i never touch HBM unless final logits are requested.
 #include <cstdint>
 
@@ -40,6 +41,8 @@ constexpr int NCW = 4;                       // consumer warps
 constexpr int NTHREADS = (NCW + 1) * 32;     // + one producer warp
 constexpr int CONS_THREADS = NCW * 32;
 constexpr uint32_t BAR_CONS = 1;             // named barrier id among consumer warps
+constexpr int L2_AHEAD = 16;                 // items prefetched into L2 ahead of the ring
+constexpr int VCHUNK = 32;                   // W2 rows per ring item
 
 struct Partition {
   int j0, j1;  // GRU units
@@ -62,17 +65,16 @@ __device__ __host__ __forceinline__ long long vend_raw(const LoopArgs& a, int c,
   return v;
 }
 
-__device__ __forceinline__ Partition partition_of(const LoopArgs& a, int c, int G) {
+// Units and bottleneck rows split evenly; the vocabulary split (computed once
+// on the host into a.vsplit) balances the weight bytes every CTA streams.
+__device__ __host__ __forceinline__ Partition partition_of(const LoopArgs& a, int c, int G) {
   Partition p;
   p.j0 = c * a.H / G;
   p.j1 = (c + 1) * a.H / G;
   p.k0 = c * a.r / G;
   p.k1 = (c + 1) * a.r / G;
-  long long lo = 0;
-  for (int cc = 0; cc < c; ++cc) lo = max(lo, vend_raw(a, cc, G));
-  const long long hi = max(lo, vend_raw(a, c, G));
-  p.v0 = static_cast<int>(lo);
-  p.v1 = static_cast<int>(hi);
+  p.v0 = a.vsplit[c];
+  p.v1 = a.vsplit[c + 1];
   return p;
 }
 
@@ -91,16 +93,17 @@ struct Shared {
   uint8_t* ring;
   float* S;        // [NB][H]   S_{i-1} (whole vector, all requests)
   uint8_t* x;      // [NB][E]   embedding of the fed token, storage type
-  float* u;        // [NB][r]
+  float* base;     // [NB][vmax] this CTA's slice of the step's base logits
   float* part;     // [max_part][32] per-item partial sums
   float* hp;       // [kmax][NB][K] W1_h h terms of this CTA's rows
+  float* bias;     // [umax][6] b_ih r,z,n then b_hh r,z,n of this CTA's units
   int* tok;        // [NB][K] picks (CTA 0 verifies from here)
   uint64_t* wbest; // [NCW][NB]
   int* flags;      // [0] abort
   int* fed;        // [NB] token fed to the GRU at the next step
+  uint8_t* items;  // [max_items] per-step ring item table (producer)
 };
 
-template <int NB>
 __device__ __forceinline__ Shared carve(uint8_t* base, const LoopArgs& a) {
   Shared s;
   s.ring = base;
@@ -108,13 +111,15 @@ __device__ __forceinline__ Shared carve(uint8_t* base, const LoopArgs& a) {
   s.empty = s.full + a.nslot;
   s.S = reinterpret_cast<float*>(base + a.off_S);
   s.x = base + a.off_x;
-  s.u = reinterpret_cast<float*>(base + a.off_u);
+  s.base = reinterpret_cast<float*>(base + a.off_base);
   s.part = reinterpret_cast<float*>(base + a.off_part);
   s.hp = reinterpret_cast<float*>(base + a.off_hp);
+  s.bias = reinterpret_cast<float*>(base + a.off_bias);
   s.tok = reinterpret_cast<int*>(base + a.off_tok);
   s.wbest = reinterpret_cast<uint64_t*>(base + a.off_wbest);
   s.flags = reinterpret_cast<int*>(base + a.off_flags);
   s.fed = s.flags + 4;
+  s.items = base + a.off_items;
   return s;
 }
 
@@ -125,12 +130,12 @@ __device__ __forceinline__ void set_abort(const Shared& s) {
   *reinterpret_cast<volatile int*>(&s.flags[0]) = 1;
 }
 
-// Consumer-wide grid barrier: named barrier, one thread arrives and waits,
-// named barrier.  Keeps control flow uniform even after an abort.
-__device__ __forceinline__ void consumer_grid_sync(const LoopArgs& a, const Shared& s, uint32_t nblocks) {
+// Consumer-wide grid barrier number k: named barrier, one thread arrives and
+// waits, named barrier.  Keeps control flow uniform even after an abort.
+__device__ __forceinline__ void consumer_grid_sync(const LoopArgs& a, const Shared& s, uint32_t k) {
   named_barrier(BAR_CONS, CONS_THREADS);
   if (threadIdx.x == 0 && !aborted(s)) {
-    if (!grid_barrier_one_thread(a.ctl, nblocks, a.budget_ns)) set_abort(s);
+    if (!grid_barrier_one_thread(a.ctl, gridDim.x * (k + 1), a.budget_ns)) set_abort(s);
   }
   named_barrier(BAR_CONS, CONS_THREADS);
 }
@@ -149,83 +154,105 @@ __device__ __forceinline__ Sched make_sched(const LoopArgs& a, int c, int G) {
   s.h1 = Seg{a.nsegH1, a.segH1};
   s.nA = (s.p.j1 - s.p.j0) * (s.e3.n + s.h3.n);
   s.nB = (s.p.k1 - s.p.k0) * s.h1.n;
-  s.nC = (s.p.v1 - s.p.v0 + 31) / 32;
+  s.nC = (s.p.v1 - s.p.v0 + VCHUNK - 1) / VCHUNK;
   s.per_step = s.nA + s.nB + s.nC;
   return s;
 }
 
+// Source ranges of ring item n: `ncopy` copies of `bytes` each (3 gate rows of
+// one unit, one W1 row segment, or one W2 row chunk).
+struct Item {
+  const uint8_t* src[3];
+  uint32_t bytes;
+  int ncopy;
+};
+__device__ __forceinline__ Item item_of(const LoopArgs& a, const Sched& sc, int n) {
+  Item it;
+  int q = n % sc.per_step;
+  const int wb = a.wbytes;
+  if (q < sc.nA) {
+    const int per_unit = sc.e3.n + sc.h3.n;
+    const int j = sc.p.j0 + q / per_unit;
+    const int s_all = q % per_unit;
+    const bool hh = s_all >= sc.e3.n;
+    const int s = hh ? s_all - sc.e3.n : s_all;
+    const Seg sg = hh ? sc.h3 : sc.e3;
+    const int ncol = hh ? a.H : a.E;
+    const uint8_t* m = static_cast<const uint8_t*>(hh ? a.w_hh : a.w_ih);
+    const int c0 = s * sg.len, len = seg_len(sg, ncol, s);
+    it.bytes = static_cast<uint32_t>(len) * wb;
+    it.ncopy = 3;
+    for (int g = 0; g < 3; ++g) it.src[g] = m + ((static_cast<size_t>(g) * a.H + j) * ncol + c0) * wb;
+    return it;
+  }
+  q -= sc.nA;
+  if (q < sc.nB) {
+    const int k = sc.p.k0 + q / sc.h1.n, s = q % sc.h1.n;
+    const int c0 = s * sc.h1.len, len = seg_len(sc.h1, a.H, s);
+    it.bytes = static_cast<uint32_t>(len) * wb;
+    it.ncopy = 1;
+    it.src[0] = static_cast<const uint8_t*>(a.w1) + (static_cast<size_t>(k) * (a.d + a.H) + a.d + c0) * wb;
+    it.src[1] = it.src[2] = nullptr;
+    return it;
+  }
+  q -= sc.nB;
+  const int v = sc.p.v0 + q * VCHUNK;
+  const int rows = min(VCHUNK, sc.p.v1 - v);
+  it.bytes = static_cast<uint32_t>(rows) * a.r * wb;
+  it.ncopy = 1;
+  it.src[0] = static_cast<const uint8_t*>(a.w2) + static_cast<size_t>(v) * a.r * wb;
+  it.src[1] = it.src[2] = nullptr;
+  return it;
+}
+
 // ---------------------------------------------------------------- producer
-template <typename W>
+// The per-step item sequence is identical for every step, so the producer
+// decodes it once into shared memory and then only walks the table.
 __device__ void producer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
   if ((threadIdx.x & 31) != 0) return;
-  const W* w_ih = static_cast<const W*>(a.w_ih);
-  const W* w_hh = static_cast<const W*>(a.w_hh);
-  const W* w1 = static_cast<const W*>(a.w1);
-  const W* w2 = static_cast<const W*>(a.w2);
+  Item* table = reinterpret_cast<Item*>(sh.items);
+  for (int q = 0; q < sc.per_step; ++q) table[q] = item_of(a, sc, q);
   const uint64_t pol = policy_evict_first();
   const int nslot = a.nslot;
-  const uint32_t slot_bytes = kLoopSlotBytes;
-  int n = 0;
-  bool ok = true;
-  auto acquire = [&](int item) -> uint8_t* {
-    const int slot = item % nslot;
-    if (item >= nslot) {
-      const uint32_t par = ((item / nslot) - 1) & 1;
-      // wait for the consumer to release the slot; give up on abort
+  const int total = a.K * sc.per_step;
+  // warm L2 with the first items
+  int ahead_q = 0;
+  for (int p = 0; p < L2_AHEAD && p < total; ++p) {
+    const Item& it = table[ahead_q];
+    for (int c = 0; c < it.ncopy; ++c) bulk_prefetch_l2(it.src[c], it.bytes);
+    if (++ahead_q == sc.per_step) ahead_q = 0;
+  }
+  int n = 0, q = 0, slot = 0;
+  uint32_t phase = 0;
+  for (; n < total; ++n) {
+    if (n >= nslot) {
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(&sh.empty[slot], par)) {
-        if (aborted(sh)) return nullptr;
+      bool ok = true;
+      while (!mbar_try_wait(&sh.empty[slot], phase ^ 1u)) {
+        if (aborted(sh)) { ok = false; break; }
         if (globaltimer_ns() - t0 > a.budget_ns) {
           raise_error(a.ctl, ERRBIT_TIMEOUT);
           set_abort(sh);
-          return nullptr;
+          ok = false;
+          break;
         }
       }
+      if (!ok) break;
     }
-    return sh.ring + static_cast<size_t>(slot) * slot_bytes;
-  };
-  for (int step = 0; step < a.K && ok; ++step) {
-    // phase A: GRU gate-row triples, input side then recurrent side
-    for (int j = sc.p.j0; j < sc.p.j1 && ok; ++j) {
-      for (int side = 0; side < 2 && ok; ++side) {
-        const W* m = side == 0 ? w_ih : w_hh;
-        const int ncol = side == 0 ? a.E : a.H;
-        const Seg sg = side == 0 ? sc.e3 : sc.h3;
-        for (int s = 0; s < sg.n; ++s, ++n) {
-          uint8_t* dst = acquire(n);
-          if (!dst) { ok = false; break; }
-          const int c0 = s * sg.len, len = seg_len(sg, ncol, s);
-          const uint32_t rowb = static_cast<uint32_t>(len) * sizeof(W);
-          mbar_arrive_expect_tx(&sh.full[n % nslot], 3u * rowb);
-          for (int g = 0; g < 3; ++g)
-            bulk_g2s(dst + g * rowb, m + (static_cast<size_t>(g) * a.H + j) * ncol + c0, rowb, &sh.full[n % nslot], pol);
-        }
-      }
+    if (n + L2_AHEAD < total) {
+      const Item& ah = table[ahead_q];
+      for (int c = 0; c < ah.ncopy; ++c) bulk_prefetch_l2(ah.src[c], ah.bytes);
+      if (++ahead_q == sc.per_step) ahead_q = 0;
     }
-    // phase B: recurrent block of W1 rows
-    for (int k = sc.p.k0; k < sc.p.k1 && ok; ++k) {
-      for (int s = 0; s < sc.h1.n; ++s, ++n) {
-        uint8_t* dst = acquire(n);
-        if (!dst) { ok = false; break; }
-        const int c0 = s * sc.h1.len, len = seg_len(sc.h1, a.H, s);
-        const uint32_t rowb = static_cast<uint32_t>(len) * sizeof(W);
-        mbar_arrive_expect_tx(&sh.full[n % nslot], rowb);
-        bulk_g2s(dst, w1 + static_cast<size_t>(k) * (a.d + a.H) + a.d + c0, rowb, &sh.full[n % nslot], pol);
-      }
-    }
-    // phase C: W2 row chunks of 32 rows
-    for (int v = sc.p.v0; v < sc.p.v1 && ok; v += 32, ++n) {
-      uint8_t* dst = acquire(n);
-      if (!dst) { ok = false; break; }
-      const int rows = min(32, sc.p.v1 - v);
-      const uint32_t bytes = static_cast<uint32_t>(rows) * a.r * sizeof(W);
-      mbar_arrive_expect_tx(&sh.full[n % nslot], bytes);
-      bulk_g2s(dst, w2 + static_cast<size_t>(v) * a.r, bytes, &sh.full[n % nslot], pol);
-    }
+    const Item& it = table[q];
+    uint8_t* dst = sh.ring + static_cast<size_t>(slot) * kLoopSlotBytes;
+    mbar_arrive_expect_tx(&sh.full[slot], it.bytes * it.ncopy);
+    for (int c = 0; c < it.ncopy; ++c) bulk_g2s(dst + c * it.bytes, it.src[c], it.bytes, &sh.full[slot], pol);
+    if (++q == sc.per_step) q = 0;
+    if (++slot == nslot) { slot = 0; phase ^= 1u; }
   }
   // drain: every issued copy must land before the CTA may exit
-  const int first = max(0, n - nslot);
-  for (int item = first; item < n; ++item) {
+  for (int item = max(0, n - nslot); item < n; ++item) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(&sh.full[item % nslot], (item / nslot) & 1)) {
       if (globaltimer_ns() - t0 > a.budget_ns) {
@@ -257,36 +284,45 @@ __device__ __forceinline__ void consume_end(const LoopArgs& a, const Shared& sh,
   if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.empty[n % a.nslot]);
 }
 
+template <typename W>
+__device__ __forceinline__ void gather_rows(const LoopArgs& a, const Shared& sh, int nrows) {
+  const W* embed = static_cast<const W*>(a.embed);
+  const int xg = a.E / 8;  // 8-element groups per embedding row
+  for (int q = threadIdx.x; q < nrows * xg; q += CONS_THREADS) {
+    const int b = q / xg, g = q % xg;
+    const W* src = embed + static_cast<size_t>(sh.fed[b]) * a.E + g * 8;
+    if (sizeof(W) == 2) {
+      reinterpret_cast<uint4*>(sh.x)[q] = __ldg(reinterpret_cast<const uint4*>(src));
+    } else {
+      reinterpret_cast<uint4*>(sh.x)[2 * q] = __ldg(reinterpret_cast<const uint4*>(src));
+      reinterpret_cast<uint4*>(sh.x)[2 * q + 1] = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    }
+  }
+}
+
 template <typename W, int NB>
 __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int G = gridDim.x;
   const bool cta0 = blockIdx.x == 0;
   const int nb = a.nb;
   const int K = a.K;
-  const W* embed = static_cast<const W*>(a.embed);
-  const W* hidden = static_cast<const W*>(a.hidden);
-  const W* w1 = static_cast<const W*>(a.w1);
   const int kmine = sc.p.k1 - sc.p.k0;
+  const int umine = sc.p.j1 - sc.p.j0;
+  const int vrows = sc.p.v1 - sc.p.v0;
+  uint32_t nbar = 0;
 
-  // ---- prologue: zero argmax keys, W1_h h_i for own rows, S = 0, first GRU input
+  // ---- prologue: argmax keys, biases, precomputed W1_h h terms, S = 0, first GRU input
   if (cta0)
     for (int q = tid; q < K * NB; q += CONS_THREADS) a.best[q] = 0ull;
-  for (int q = warp; q < kmine * nb * K; q += NCW) {
+  for (int q = tid; q < umine * 6; q += CONS_THREADS) {
+    const int jl = q / 6, g = q % 6;
+    const float* bsrc = g < 3 ? a.b_ih : a.b_hh;
+    sh.bias[q] = bsrc ? bsrc[(g % 3) * a.H + sc.p.j0 + jl] : 0.f;
+  }
+  for (int q = tid; q < kmine * nb * K; q += CONS_THREADS) {
     const int kl = q / (nb * K), rem = q % (nb * K), b = rem / K, p = rem % K;
-    const W* wrow = w1 + static_cast<size_t>(sc.p.k0 + kl) * (a.d + a.H);
-    const W* hrow = hidden + (static_cast<size_t>(b) * K + p) * a.d;
-    float acc = 0.f;
-    for (int g = lane; g < a.d / 8; g += 32) {
-      float wv[8], hv[8];
-      widen8(wrow + g * 8, wv);
-      widen8(hrow + g * 8, hv);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc = fmaf(wv[e], hv[e], acc);
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) sh.hp[(kl * NB + b) * K + p] = acc;
+    sh.hp[(kl * NB + b) * K + p] = a.hp[(static_cast<size_t>(b) * K + p) * a.r + sc.p.k0 + kl];
   }
   for (int q = tid; q < NB * a.H; q += CONS_THREADS) sh.S[q] = 0.f;
   if (tid < NB) {
@@ -298,24 +334,21 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     sh.fed[tid] = t;
   }
   named_barrier(BAR_CONS, CONS_THREADS);
-  const int xg = a.E / 8;  // 8-element groups per embedding row
-  for (int q = tid; q < NB * xg; q += CONS_THREADS) {
-    const int b = q / xg, g = q % xg;
-    const uint4 v = *reinterpret_cast<const uint4*>(embed + static_cast<size_t>(sh.fed[b]) * a.E + g * 8);
-    // storage widths: bf16 -> 16 B per group; f32 -> 32 B per group
-    if (sizeof(W) == 2) {
-      reinterpret_cast<uint4*>(sh.x)[q] = v;
-    } else {
-      const uint4 v2 = *reinterpret_cast<const uint4*>(embed + static_cast<size_t>(sh.fed[b]) * a.E + g * 8 + 4);
-      reinterpret_cast<uint4*>(sh.x)[2 * q] = v;
-      reinterpret_cast<uint4*>(sh.x)[2 * q + 1] = v2;
-    }
-  }
+  gather_rows<W>(a, sh, NB);
   named_barrier(BAR_CONS, CONS_THREADS);
 
   int n_base = 0;  // global item index of the first item of the current phase
 
   for (int i = 0; i < K; ++i) {
+    // base-logit slice of this step -> shared memory, overlapped with the GRU
+    if (!aborted(sh)) {
+      for (int q = tid; q < nb * vrows; q += CONS_THREADS) {
+        const int b = q / vrows, v = q % vrows;
+        cp_async4(sh.base + b * a.vmax + v, a.base + (static_cast<size_t>(b) * K + i) * a.V + sc.p.v0 + v);
+      }
+    }
+    cp_async_commit();
+
     // ================= phase A: GRU partial dot products
     for (int q = 0; q < sc.nA; ++q) {
       const int n = n_base + q;
@@ -369,18 +402,18 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     float* S_new = a.S_glob + static_cast<size_t>((i + 1) & 1) * NB * a.H;
     if (!aborted(sh)) {
       const int per_unit = sc.e3.n + sc.h3.n;
-      for (int q = tid; q < (sc.p.j1 - sc.p.j0) * NB; q += CONS_THREADS) {
+      for (int q = tid; q < umine * NB; q += CONS_THREADS) {
         const int jl = q / NB, b = q % NB;
         const int j = sc.p.j0 + jl;
-        float gi[3] = {0.f, 0.f, 0.f}, gh[3] = {0.f, 0.f, 0.f};
+        float gi[3], gh[3];
+        for (int g = 0; g < 3; ++g) {
+          gi[g] = sh.bias[jl * 6 + g];
+          gh[g] = sh.bias[jl * 6 + 3 + g];
+        }
         for (int s = 0; s < sc.e3.n; ++s)
           for (int g = 0; g < 3; ++g) gi[g] += sh.part[(jl * per_unit + s) * 32 + g * NB + b];
         for (int s = 0; s < sc.h3.n; ++s)
           for (int g = 0; g < 3; ++g) gh[g] += sh.part[(jl * per_unit + sc.e3.n + s) * 32 + g * NB + b];
-        for (int g = 0; g < 3; ++g) {
-          gi[g] += a.b_ih ? a.b_ih[g * a.H + j] : 0.f;
-          gh[g] += a.b_hh ? a.b_hh[g * a.H + j] : 0.f;
-        }
         const float r = 1.f / (1.f + expf(-(gi[0] + gh[0])));
         const float z = 1.f / (1.f + expf(-(gi[1] + gh[1])));
         const float nn = tanhf(gi[2] + r * gh[2]);
@@ -388,7 +421,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
         S_new[b * a.H + j] = (1.f - z) * nn + z * s_old;
       }
     }
-    consumer_grid_sync(a, sh, G);  // ---- barrier 1: S_i complete
+    consumer_grid_sync(a, sh, nbar++);  // ---- barrier 1: S_i complete
 
     // S_i -> shared (L1 bypassed: other SMs wrote it)
     if (!aborted(sh)) {
@@ -434,7 +467,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
         a.u_glob[b * a.r + sc.p.k0 + kl] = silu;
       }
     }
-    consumer_grid_sync(a, sh, G);  // ---- barrier 2: u complete
+    consumer_grid_sync(a, sh, nbar++);  // ---- barrier 2: u complete
 
     // u -> registers: lane holds u[b][8*lane .. 8*lane+8)
     float ureg[NB][8];
@@ -453,6 +486,8 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
         }
       }
     }
+    cp_async_wait_all();
+    named_barrier(BAR_CONS, CONS_THREADS);
 
     // ================= phase C: W2 chunks, residual, pick
     constexpr int RPI = 32 / NB;           // rows per reduce-scatter round
@@ -463,17 +498,8 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     for (int q = 0; q < sc.nC; ++q) {
       const int n = n_base + q;
       if (n % NCW != warp) continue;
-      const int vstart = sc.p.v0 + q * 32;
-      const int rows = min(32, sc.p.v1 - vstart);
-      // prefetch base logits for the (row, request) pairs this lane finalises
-      float bpre[NB];
-#pragma unroll
-      for (int it = 0; it < NB; ++it) {
-        const int rl = it * RPI + lane / NB;
-        bpre[it] = (rl < rows && my_b < nb)
-                       ? __ldg(a.base + (static_cast<size_t>(my_b) * K + i) * a.V + vstart + rl)
-                       : 0.f;
-      }
+      const int vl0 = q * VCHUNK;          // chunk start, relative to v0
+      const int rows = min(VCHUNK, vrows - vl0);
       const uint8_t* slot = consume_begin(a, sh, n);
       if (slot) {
 #pragma unroll
@@ -498,8 +524,8 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
           const float dl = warp_reduce_scatter32(acc);
           const int rl = it * RPI + lane / NB;
           if (rl < rows && my_b < nb) {
-            const int v = vstart + rl;
-            const float L = bpre[it] + dl;
+            const int v = sc.p.v0 + vl0 + rl;
+            const float L = sh.base[my_b * a.vmax + vl0 + rl] + dl;
             if (a.logits) a.logits[(static_cast<size_t>(my_b) * K + i) * a.V + v] = L;
             float score = L;
             if (!greedy) score = __fdiv_rn(L, a.temperature) + gumbel_noise(a.seed, a.b0 + my_b, i, v);
@@ -524,7 +550,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       for (int w = 0; w < NCW; ++w) k = max(k, sh.wbest[w * NB + tid]);
       if (k != 0ull) atomicMax(reinterpret_cast<unsigned long long*>(&a.best[i * NB + tid]), static_cast<unsigned long long>(k));
     }
-    consumer_grid_sync(a, sh, G);  // ---- barrier 3: picks merged
+    consumer_grid_sync(a, sh, nbar++);  // ---- barrier 3: picks merged
 
     // picks, next GRU input
     if (tid < nb) {
@@ -541,19 +567,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       sh.fed[b] = f;
     }
     named_barrier(BAR_CONS, CONS_THREADS);
-    if (i + 1 < K && !aborted(sh)) {
-      for (int q = tid; q < nb * xg; q += CONS_THREADS) {
-        const int b = q / xg, g = q % xg;
-        const uint4 v = *reinterpret_cast<const uint4*>(embed + static_cast<size_t>(sh.fed[b]) * a.E + g * 8);
-        if (sizeof(W) == 2) {
-          reinterpret_cast<uint4*>(sh.x)[q] = v;
-        } else {
-          const uint4 v2 = *reinterpret_cast<const uint4*>(embed + static_cast<size_t>(sh.fed[b]) * a.E + g * 8 + 4);
-          reinterpret_cast<uint4*>(sh.x)[2 * q] = v;
-          reinterpret_cast<uint4*>(sh.x)[2 * q + 1] = v2;
-        }
-      }
-    }
+    if (i + 1 < K && !aborted(sh)) gather_rows<W>(a, sh, nb);
     named_barrier(BAR_CONS, CONS_THREADS);
   }
 
@@ -565,31 +579,34 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       a.tau[b] = t;
     }
   }
+  if (tid == 0) grid_exit(a.ctl, gridDim.x);
 }
 
 template <typename W, int NB>
 __global__ void __launch_bounds__(NTHREADS, 1) correct_loop_kernel(const LoopArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  Shared sh = carve<NB>(smem, a);
   const int G = gridDim.x;
   if (a.selftest) {
     // one barrier episode that can never complete: exercises the bounded wait
-    if (threadIdx.x == 0) grid_barrier_one_thread(a.ctl, static_cast<uint32_t>(G) + 1u, a.budget_ns);
+    if (threadIdx.x == 0) {
+      grid_barrier_one_thread(a.ctl, static_cast<uint32_t>(G) + 1u, a.budget_ns);
+      grid_exit(a.ctl, G);
+    }
     return;
   }
+  Shared sh = carve(smem, a);
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.nslot; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
     sh.flags[0] = 0;
-    sh.flags[1] = 0;
     fence_mbar_init();
   }
   __syncthreads();
   const Sched sc = make_sched(a, blockIdx.x, G);
   if (threadIdx.x >= CONS_THREADS) {
-    producer<W>(a, sh, sc);
+    producer(a, sh, sc);
   } else {
     consumer<W, NB>(a, sh, sc);
   }
@@ -626,45 +643,53 @@ size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap) {
   const int kmax = (a.r + grid - 1) / grid;
   a.max_part = umax * (a.nsegE3 + a.nsegH3);
   a.max_part = a.max_part > kmax * a.nsegH1 ? a.max_part : kmax * a.nsegH1;
-  size_t off = 0;
-  auto take = [&](size_t bytes, size_t align) {
-    off = (off + align - 1) / align * align;
-    const size_t at = off;
-    off += bytes;
-    return static_cast<uint32_t>(at);
-  };
-  // everything except the ring first, then as many slots as fit (multiple of NCW)
-  size_t fixed = 0;
-  {
-    size_t o = 0;
-    auto t2 = [&](size_t bytes, size_t align) { o = (o + align - 1) / align * align; o += bytes; };
-    t2(2 * 8 * 64, 8);
-    t2(static_cast<size_t>(NB) * a.H * 4, 16);
-    t2(static_cast<size_t>(NB) * a.E * wb, 16);
-    t2(static_cast<size_t>(NB) * a.r * 4, 16);
-    t2(static_cast<size_t>(a.max_part) * 32 * 4, 16);
-    t2(static_cast<size_t>(kmax) * NB * a.K * 4, 16);
-    t2(static_cast<size_t>(NB) * a.K * 4, 16);
-    t2(static_cast<size_t>(NCW) * NB * 8, 8);
-    t2(64, 16);
-    fixed = o + 1024;
+  if (grid > kLoopMaxGrid) return 0;
+  // vocabulary split: running maximum of the byte-balanced cut points
+  long long lo = 0;
+  a.vsplit[0] = 0;
+  for (int c = 0; c < grid; ++c) {
+    const long long raw = vend_raw(a, c, grid);
+    lo = lo > raw ? lo : raw;
+    a.vsplit[c + 1] = static_cast<int32_t>(lo);
   }
+  a.vsplit[grid] = a.V;
+  int vmax = 0, items_max = 0;
+  for (int c = 0; c < grid; ++c) {
+    const Partition p = partition_of(a, c, grid);
+    vmax = vmax > p.v1 - p.v0 ? vmax : p.v1 - p.v0;
+    const int n = (p.j1 - p.j0) * (a.nsegE3 + a.nsegH3) + (p.k1 - p.k0) * a.nsegH1 + (p.v1 - p.v0 + VCHUNK - 1) / VCHUNK;
+    items_max = items_max > n ? items_max : n;
+  }
+  a.vmax = (vmax + 3) / 4 * 4;
+  struct Piece { uint32_t* off; size_t bytes; size_t align; };
+  const Piece pieces[] = {
+      {&a.off_S, static_cast<size_t>(NB) * a.H * 4, 16},
+      {&a.off_x, static_cast<size_t>(NB) * a.E * wb, 16},
+      {&a.off_base, static_cast<size_t>(NB) * a.vmax * 4, 16},
+      {&a.off_part, static_cast<size_t>(a.max_part) * 32 * 4, 16},
+      {&a.off_hp, static_cast<size_t>(kmax) * NB * a.K * 4, 16},
+      {&a.off_bias, static_cast<size_t>(umax) * 6 * 4, 16},
+      {&a.off_tok, static_cast<size_t>(NB) * a.K * 4, 16},
+      {&a.off_wbest, static_cast<size_t>(NCW) * NB * 8, 8},
+      {&a.off_flags, 64, 16},
+      {&a.off_items, static_cast<size_t>(items_max) * sizeof(Item), 16},
+  };
+  size_t fixed = 2 * 8 * 16 + 16;  // barriers of up to 16 slots
+  for (const Piece& p : pieces) fixed = (fixed + p.align - 1) / p.align * p.align + p.bytes;
+  fixed += 1024;
   if (fixed >= smem_cap) return 0;
   int nslot = static_cast<int>((smem_cap - fixed) / kLoopSlotBytes) / NCW * NCW;
   if (nslot > 16) nslot = 16;
   if (nslot < NCW) return 0;
   a.nslot = nslot;
-  off = 0;
-  take(static_cast<size_t>(nslot) * kLoopSlotBytes, 1024);
-  a.off_bars = take(2 * 8 * nslot, 8);
-  a.off_S = take(static_cast<size_t>(NB) * a.H * 4, 16);
-  a.off_x = take(static_cast<size_t>(NB) * a.E * wb, 16);
-  a.off_u = take(static_cast<size_t>(NB) * a.r * 4, 16);
-  a.off_part = take(static_cast<size_t>(a.max_part) * 32 * 4, 16);
-  a.off_hp = take(static_cast<size_t>(kmax) * NB * a.K * 4, 16);
-  a.off_tok = take(static_cast<size_t>(NB) * a.K * 4, 16);
-  a.off_wbest = take(static_cast<size_t>(NCW) * NB * 8, 8);
-  a.off_flags = take(64, 16);
+  size_t off = static_cast<size_t>(nslot) * kLoopSlotBytes;
+  a.off_bars = static_cast<uint32_t>(off);
+  off += 2 * 8 * nslot;
+  for (const Piece& p : pieces) {
+    off = (off + p.align - 1) / p.align * p.align;
+    *p.off = static_cast<uint32_t>(off);
+    off += p.bytes;
+  }
   return off;
 }
 

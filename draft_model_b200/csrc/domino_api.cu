@@ -6,7 +6,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "../../include/domino.h"
+#include "domino.h"
 #include "common.cuh"
 #include "domino_internal.h"
 
@@ -30,7 +30,7 @@ int num_sms() {
 }
 
 struct Layout {
-  size_t ctl, base, S, u, best, end;                       // device workspace
+  size_t ctl, base, hp, S, u, best, end;                   // device workspace
   size_t h_hidden, h_anchor, h_forced, h_target, h_draft, h_tau, h_end;  // host-variant staging
 };
 
@@ -60,6 +60,7 @@ Layout layout_of(const domino_weights* w, int B, int K) {
   size_t o = 0;
   L.ctl = o; o += align_up(sizeof(Control));
   L.base = o; o += align_up(static_cast<size_t>(B) * K * w->vocab * 4);
+  L.hp = o; o += align_up(static_cast<size_t>(B) * K * w->rank * 4);
   L.S = o; o += align_up(2ull * 8 * w->gru_hidden * 4);
   L.u = o; o += align_up(8ull * w->rank * 4);
   L.best = o; o += align_up(static_cast<size_t>(K) * 8 * 8);
@@ -86,17 +87,24 @@ domino_status check_workspace(void* ws, size_t bytes, size_t need) {
   return DOMINO_OK;
 }
 
-domino_status run_lm_head(const domino_weights* w, const void* hidden, int B, int K, float* base, Control* ctl,
-                          cudaStream_t st) {
+// Stage 1: base logits (base != null) and/or the hidden-state half of the
+// bottleneck pre-activation hp[m, k] = W1[k, 0:d] h[m] (hp != null).
+domino_status run_lm_head(const domino_weights* w, const void* hidden, int B, int K, float* base, float* hp,
+                          Control* ctl, cudaStream_t st) {
   const int M = B * K;
-  cudaError_t e;
+  const int w1_stride = w->d_model + w->gru_hidden;
+  cudaError_t e = cudaSuccess;
   if (w->dtype == DOMINO_BF16) {
     const int sms = num_sms();
     if (sms <= 0) return DOMINO_ERR_CUDA;
-    e = domino::launch_lm_head_tc(w->w_lm, hidden, base, w->vocab, M, w->d_model, ctl, g_budget_ns.load(), sms, st);
+    e = domino::launch_lm_head_tc(w->w_lm, hidden, base, w->vocab, M, w->d_model, w->w1, w->rank, w1_stride, hp, ctl,
+                                  g_budget_ns.load(), sms, st);
   } else {
-    e = domino::launch_lm_head_f32(static_cast<const float*>(w->w_lm), static_cast<const float*>(hidden), base,
-                                   w->vocab, M, w->d_model, st);
+    const float* h = static_cast<const float*>(hidden);
+    if (base) e = domino::launch_lm_head_f32(static_cast<const float*>(w->w_lm), h, base, w->vocab, M, w->d_model,
+                                             w->d_model, st);
+    if (e == cudaSuccess && hp)
+      e = domino::launch_lm_head_f32(static_cast<const float*>(w->w1), h, hp, w->rank, M, w->d_model, w1_stride, st);
   }
   return from_cuda(e);
 }
@@ -121,6 +129,7 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
   a.ctl = reinterpret_cast<Control*>(ws + L.ctl);
   a.S_glob = reinterpret_cast<float*>(ws + L.S);
   a.u_glob = reinterpret_cast<float*>(ws + L.u);
+  const float* hp = reinterpret_cast<const float*>(ws + L.hp);
   a.best = reinterpret_cast<unsigned long long*>(ws + L.best);
   a.seed = seed;
   a.budget_ns = g_budget_ns.load();
@@ -142,6 +151,7 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
     g.nb = nb;
     g.hidden = static_cast<const char*>(hidden) + static_cast<size_t>(g0) * K * w->d_model * wb;
     g.base = base + static_cast<size_t>(g0) * K * w->vocab;
+    g.hp = hp + static_cast<size_t>(g0) * K * w->rank;
     g.anchor = anchor + g0;
     g.forced = forced ? forced + static_cast<size_t>(g0) * K : nullptr;
     g.target = target ? target + static_cast<size_t>(g0) * K : nullptr;
@@ -198,7 +208,8 @@ domino_status domino_lm_head(const domino_weights* w, const void* hidden, int32_
     return DOMINO_ERR_INVALID_ARG;
   const domino_status ws = check_workspace(workspace, workspace_bytes, sizeof(Control));
   if (ws != DOMINO_OK) return ws;
-  return run_lm_head(w, hidden, B, K, base_out, static_cast<Control*>(workspace), static_cast<cudaStream_t>(stream));
+  return run_lm_head(w, hidden, B, K, base_out, nullptr, static_cast<Control*>(workspace),
+                     static_cast<cudaStream_t>(stream));
 }
 
 domino_status domino_correct_loop(const domino_weights* w, const void* hidden, const float* base,
@@ -213,14 +224,20 @@ domino_status domino_correct_loop(const domino_weights* w, const void* hidden, c
   const Layout L = layout_of(w, B, K);
   s = check_workspace(workspace, workspace_bytes, L.end);
   if (s != DOMINO_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = run_lm_head(w, hidden, B, K, nullptr, reinterpret_cast<float*>(ws + L.hp), reinterpret_cast<Control*>(ws + L.ctl),
+                  st);
+  if (s != DOMINO_OK) return s;
   return run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out,
-                  tau_out, static_cast<char*>(workspace), L, static_cast<cudaStream_t>(stream));
+                  tau_out, ws, L, st);
 }
 
-domino_status domino_draft_block(const domino_weights* w, const void* hidden, const int32_t* anchor, int32_t B,
-                                 int32_t K, int32_t mode, float temperature, uint64_t seed, const int32_t* forced,
-                                 const int32_t* target, int32_t* draft_out, float* logits_out, int32_t* tau_out,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+domino_status domino_draft_block_events(const domino_weights* w, const void* hidden, const int32_t* anchor, int32_t B,
+                                        int32_t K, int32_t mode, float temperature, uint64_t seed,
+                                        const int32_t* forced, const int32_t* target, int32_t* draft_out,
+                                        float* logits_out, int32_t* tau_out, void* workspace, size_t workspace_bytes,
+                                        void* stream, void* const* events) {
   domino_status s = validate_block(w, hidden, anchor, B, K, mode, temperature, forced, target, draft_out,
                                    logits_out, tau_out);
   if (s != DOMINO_OK) return s;
@@ -230,11 +247,28 @@ domino_status domino_draft_block(const domino_weights* w, const void* hidden, co
   if (s != DOMINO_OK) return s;
   char* ws = static_cast<char*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int k) -> domino_status {
+    if (!events || !events[k]) return DOMINO_OK;
+    return from_cuda(cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st));
+  };
+  if ((s = mark(0)) != DOMINO_OK) return s;
   float* base = reinterpret_cast<float*>(ws + L.base);
-  s = run_lm_head(w, hidden, B, K, base, reinterpret_cast<Control*>(ws + L.ctl), st);
+  s = run_lm_head(w, hidden, B, K, base, reinterpret_cast<float*>(ws + L.hp), reinterpret_cast<Control*>(ws + L.ctl),
+                  st);
   if (s != DOMINO_OK) return s;
-  return run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out,
-                  tau_out, ws, L, st);
+  if ((s = mark(1)) != DOMINO_OK) return s;
+  s = run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out, tau_out,
+               ws, L, st);
+  if (s != DOMINO_OK) return s;
+  return mark(2);
+}
+
+domino_status domino_draft_block(const domino_weights* w, const void* hidden, const int32_t* anchor, int32_t B,
+                                 int32_t K, int32_t mode, float temperature, uint64_t seed, const int32_t* forced,
+                                 const int32_t* target, int32_t* draft_out, float* logits_out, int32_t* tau_out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return domino_draft_block_events(w, hidden, anchor, B, K, mode, temperature, seed, forced, target, draft_out,
+                                   logits_out, tau_out, workspace, workspace_bytes, stream, nullptr);
 }
 
 domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K, int32_t* tau_out,

@@ -11,6 +11,8 @@ struct Control;
 
 // Bytes per slot of the correction loop's weight ring.
 constexpr uint32_t kLoopSlotBytes = 16384;
+// Largest grid the correction loop is planned for (one CTA per SM).
+constexpr int kLoopMaxGrid = 192;
 
 // Launch arguments of the persistent correction-loop kernel (one request group).
 struct LoopArgs {
@@ -25,6 +27,7 @@ struct LoopArgs {
   // inputs (already offset to the group's first request)
   const void* hidden;   // [nb, K, d]
   const float* base;    // [nb, K, V]
+  const float* hp;      // [nb, K, r]  W1[:, 0:d] h terms (stage-1 output)
   const int32_t* anchor;
   const int32_t* forced;  // or null
   const int32_t* target;  // or null
@@ -50,8 +53,10 @@ struct LoopArgs {
   int32_t segE3, nsegE3, segH3, nsegH3, segH1, nsegH1;
   int32_t max_part;
   int32_t nslot;
+  int32_t vmax;     // largest vocabulary slice of any CTA (rounded up to 4)
+  int32_t vsplit[kLoopMaxGrid + 1];  // CTA c owns W2 rows [vsplit[c], vsplit[c+1])
   // shared-memory carve-up (byte offsets)
-  uint32_t off_bars, off_S, off_x, off_u, off_part, off_hp, off_tok, off_wbest, off_flags;
+  uint32_t off_bars, off_S, off_x, off_base, off_part, off_hp, off_bias, off_tok, off_wbest, off_flags, off_items;
 };
 
 // Fills the segment plan and shared-memory offsets; returns the dynamic shared
@@ -62,9 +67,12 @@ int loop_threads();
 cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaStream_t stream);
 
 // LM head (stage 1).
+// out [M, V] = hidden . W_lm^T (skipped if out is null); out2 [M, rows2] =
+// hidden . W1[:, 0:Kd]^T with W1 rows w1_stride elements apart (skipped if null).
 cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd,
-                              Control* ctl, uint64_t budget_ns, int num_sms, cudaStream_t stream);
-cudaError_t launch_lm_head_f32(const float* w_lm, const float* hidden, float* out, int V, int M, int Kd,
+                              const void* w1, int rows2, int w1_stride, float* out2, Control* ctl,
+                              uint64_t budget_ns, int num_sms, cudaStream_t stream);
+cudaError_t launch_lm_head_f32(const float* w, const float* hidden, float* out, int V, int M, int Kd, int ldw,
                                cudaStream_t stream);
 
 // Verification (stage 3).

@@ -1,7 +1,10 @@
 // Stage 1 of the Domino draft block on the tcgen05 tensor cores (sm_100a):
 // base logits L^base[m, v] = sum_k W_lm[v, k] h[m, k] for every block position m
 // (m = b*K + i), computed once per block (Domino study notes, gsyq.cn, §二.1(1);
-// yhxrc.cn article, §三 第一个阶段).
+// yhxrc.cn article, §三 第一个阶段).  The same launch also produces the
+// hidden-state half of the bottleneck pre-activation, P[m, k] = W1[k, 0:d] h[m]
+// (yhxrc.cn §四: W1 acts on [h_i ; S_{i-1}], and the h_i part depends on the
+// backbone only), as two extra 128-row A tiles read from W1 with its row stride.
 //
 // Swap-AB formulation: the UMMA "A" operand is a 128-row tile of W_lm (vocabulary
 // on the M side, so V = 151936 = 1187 x 128 tiles exactly) and "B" is a tile of
@@ -35,7 +38,8 @@ constexpr int NTH = 192;
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 
 struct TcArgs {
-  float* out;
+  float* out;        // [M, V]
+  float* out2;       // [M, rows2] (second A operand's products) or null
   Control* ctl;
   uint64_t budget_ns;
   int V, M, Kd;
@@ -43,6 +47,7 @@ struct TcArgs {
   int stages;
   int tmem_cols;     // power of two >= 2*BN
   int num_vt, num_mt, num_kb;
+  int rows2, num_vt2;  // second A operand: rows and 128-row tiles (0 = none)
 };
 
 // ---- tcgen05 / TMA primitives (inline PTX) ----
@@ -108,7 +113,8 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(int n) {
 }
 
 __global__ void __launch_bounds__(NTH, 1)
-    lm_head_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
+    lm_head_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                      const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment of every stage (the swizzle atom)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -124,7 +130,9 @@ __global__ void __launch_bounds__(NTH, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = a.num_vt * a.num_mt;
+  // tiles of the second A operand come first so they never land in the tail
+  const int ntiles2 = a.num_vt2 * a.num_mt;
+  const int ntiles = ntiles2 + a.num_vt * a.num_mt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -139,6 +147,7 @@ __global__ void __launch_bounds__(NTH, 1)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
+    if (a.num_vt2) prefetch_tmap(&tmA2);
     prefetch_tmap(&tmB);
   }
   if (warp == 1) tmem_alloc(tmem_slot, a.tmem_cols);
@@ -167,14 +176,17 @@ __global__ void __launch_bounds__(NTH, 1)
       int it = 0;  // global k-block counter
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int vt = t / a.num_mt, mt = t % a.num_mt;
+        const bool second = t < ntiles2;
+        const int tt = second ? t : t - ntiles2;
+        const int vt = tt / a.num_mt, mt = tt % a.num_mt;
+        const CUtensorMap* tA = second ? &tmA2 : &tmA;
         for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
           const int s = it % a.stages;
           if (it >= a.stages && !bounded_wait(&empty[s], ((it / a.stages) - 1) & 1)) { ok = false; break; }
           uint8_t* sa = smem + static_cast<size_t>(s) * stage_bytes;
           uint8_t* sb = sa + A_STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
-          tma_load_2d(sa, &tmA, kb * BK, vt * BM, &full[s]);
+          tma_load_2d(sa, tA, kb * BK, vt * BM, &full[s]);
           tma_load_2d(sb, &tmB, kb * BK, mt * a.BN, &full[s]);
         }
       }
@@ -230,8 +242,12 @@ __global__ void __launch_bounds__(NTH, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      const int vt = t / a.num_mt, mt = t % a.num_mt;
+      const bool second = t < ntiles2;
+      const int tt = second ? t : t - ntiles2;
+      const int vt = tt / a.num_mt, mt = tt % a.num_mt;
       const int v = vt * BM + q * 32 + lane;
+      const int nrows = second ? a.rows2 : a.V;
+      float* dst = second ? a.out2 : a.out;
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
       for (int c0 = 0; c0 < a.BN; c0 += 16) {
         float vals[16];
@@ -239,7 +255,7 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int m = mt * a.BN + c0 + c;
-          if (v < a.V && m < a.M) a.out[static_cast<size_t>(m) * a.V + v] = vals[c];
+          if (v < nrows && m < a.M) dst[static_cast<size_t>(m) * nrows + v] = vals[c];
         }
       }
       tc_fence_before();
@@ -271,11 +287,11 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-bool make_tmap(CUtensorMap* tm, const void* ptr, int rows, int cols, int box_rows) {
+bool make_tmap(CUtensorMap* tm, const void* ptr, int rows, int cols, int box_rows, int row_stride) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride) * 2};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -285,10 +301,13 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, int rows, int cols, int box_row
 
 }  // namespace
 
-cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd, Control* ctl,
-                              uint64_t budget_ns, int num_sms, cudaStream_t stream) {
+cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd,
+                              const void* w1, int rows2, int w1_stride, float* out2, Control* ctl, uint64_t budget_ns,
+                              int num_sms, cudaStream_t stream) {
   TcArgs a;
   a.out = out;
+  a.out2 = out2;
+  a.rows2 = out2 ? rows2 : 0;
   a.ctl = ctl;
   a.budget_ns = budget_ns;
   a.V = V;
@@ -299,7 +318,8 @@ cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, 
   int cols = 32;
   while (cols < 2 * a.BN) cols <<= 1;
   a.tmem_cols = cols;
-  a.num_vt = (V + BM - 1) / BM;
+  a.num_vt = out ? (V + BM - 1) / BM : 0;
+  a.num_vt2 = out2 ? (rows2 + BM - 1) / BM : 0;
   a.num_mt = (M + a.BN - 1) / a.BN;
   a.num_kb = (Kd + BK - 1) / BK;
   const uint32_t stage_bytes = A_STAGE_BYTES + static_cast<uint32_t>(a.BN) * BK * 2;
@@ -310,16 +330,22 @@ cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, 
   a.stages = stages;
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + 1024 /*align*/ + 256 /*barriers*/;
 
-  CUtensorMap tmA, tmB;
-  if (!make_tmap(&tmA, w_lm, V, Kd, BM)) return cudaErrorInvalidValue;
-  if (!make_tmap(&tmB, hidden, M, Kd, a.BN)) return cudaErrorInvalidValue;
+  CUtensorMap tmA, tmA2, tmB;
+  if (!make_tmap(&tmA, out ? w_lm : w1, out ? V : rows2, Kd, BM, out ? Kd : w1_stride)) return cudaErrorInvalidValue;
+  if (out2) {
+    if (!make_tmap(&tmA2, w1, rows2, Kd, BM, w1_stride)) return cudaErrorInvalidValue;
+  } else {
+    tmA2 = tmA;
+  }
+  if (!make_tmap(&tmB, hidden, M, Kd, a.BN, Kd)) return cudaErrorInvalidValue;
 
   cudaError_t e = cudaFuncSetAttribute(lm_head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int ntiles = a.num_vt * a.num_mt;
+  const int ntiles = (a.num_vt + a.num_vt2) * a.num_mt;
+  if (ntiles == 0) return cudaSuccess;
   const int grid = ntiles < num_sms ? ntiles : num_sms;
-  lm_head_tc_kernel<<<grid, NTH, smem, stream>>>(tmA, tmB, a);
+  lm_head_tc_kernel<<<grid, NTH, smem, stream>>>(tmA, tmA2, tmB, a);
   return cudaGetLastError();
 }
 

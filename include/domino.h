@@ -122,6 +122,16 @@ DOMINO_API domino_status domino_draft_block(const domino_weights* w, const void*
                                  float* logits_out, int32_t* tau_out, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* domino_draft_block that also records CUDA events on `stream` around its
+ * stages: events[0] before stage 1, events[1] between stage 1 and stage 2,
+ * events[2] after stage 2 (each a cudaEvent_t created by the caller; NULL
+ * entries are skipped).  For timing the stages of one draft block in place. */
+DOMINO_API domino_status domino_draft_block_events(const domino_weights* w, const void* hidden, const int32_t* anchor,
+                                        int32_t B, int32_t K, int32_t mode, float temperature, uint64_t seed,
+                                        const int32_t* forced, const int32_t* target, int32_t* draft_out,
+                                        float* logits_out, int32_t* tau_out, void* workspace,
+                                        size_t workspace_bytes, void* stream, void* const* events);
+
 /* Stage 1 only: base_out[b, i, v] = sum_k W_lm[v, k] hidden[b, i, k]  ([B, K, V] f32).
  * bf16 runs on the tcgen05 tensor cores, f32 on CUDA cores (no tf32). */
 DOMINO_API domino_status domino_lm_head(const domino_weights* w, const void* hidden, int32_t B, int32_t K,

@@ -12,8 +12,8 @@ zero-correction invariants; teacher-forcing and causality invariants; a
 brute-force greedy fixed point; the exact Gumbel-max law; tau by brute force;
 the head's parameter count against the pages' "56M".
 """
-from .domino_ref import Model, Result, draft_block, gru_cell, lm_head, sigmoid, silu, verify, widen_f64
+from .domino_ref import Model, Result, draft_block, gru_cell, lm_head, positions, sigmoid, silu, verify, widen_f64
 from .philox import gumbel_noise, philox4x32_10, philox4x32_10_np, uniform_from_word
 
-__all__ = ["Model", "Result", "draft_block", "gru_cell", "lm_head", "sigmoid", "silu", "verify",
+__all__ = ["Model", "Result", "draft_block", "gru_cell", "lm_head", "positions", "sigmoid", "silu", "verify",
            "widen_f64", "gumbel_noise", "philox4x32_10", "philox4x32_10_np", "uniform_from_word"]

@@ -168,6 +168,35 @@ class Result:
     tau: np.ndarray | None    # [B] acceptance length (if a target was given)
 
 
+def positions(model: Model, hidden64: np.ndarray, anchor: np.ndarray, base: np.ndarray, *,
+              mode: str = "greedy", temperature: float = 1.0, seed: int = 0,
+              forced: np.ndarray | None = None, request_ids: np.ndarray | None = None):
+    """The sequential correction loop, one block position per iteration.
+
+    Yields (p, L, score, pick) for p = 0..K-1 (block position i = p + 1): the
+    final logits L_i [B, V], the pick scores and the picks.
+    """
+    B, K, d = hidden64.shape
+    V, H = model.V, model.H
+    rid = np.arange(B) if request_ids is None else np.asarray(request_ids, dtype=np.int64)
+    s = np.zeros((B, H))
+    prev = np.asarray(anchor, dtype=np.int64).copy()
+    for p in range(K):                      # block position i = p + 1
+        x = model.embed_rows(prev)          # embedding of the token fed at this step
+        s = gru_cell(x, s, model.w_ih, model.w_hh, model.b_ih, model.b_hh)   # S_{i-1}
+        cat = np.concatenate([hidden64[:, p, :], s], axis=1)                 # [h_i ; S_{i-1}]
+        u = silu(cat @ model.w1.T)                                           # rank-r bottleneck
+        L = base[:, p, :] + u @ model.w2.T                                   # L_i = L_i^base + dL_i
+        if mode == "greedy":
+            score = L
+        else:
+            g = np.stack([gumbel_noise(seed, int(rid[b]), p + 1, V) for b in range(B)])
+            score = L / temperature + g
+        pick = np.argmax(score, axis=1)      # first index among equal maxima
+        yield p, L, score, pick
+        prev = np.asarray(forced, dtype=np.int64)[:, p] if forced is not None else pick.astype(np.int64)
+
+
 def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
                 mode: str = "greedy", temperature: float = 1.0, seed: int = 0,
                 forced: np.ndarray | None = None, target: np.ndarray | None = None,
@@ -187,7 +216,7 @@ def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
         raise ValueError("Gumbel picks need T > 0")
     h64 = widen_f64(hidden, model.dtype)
     B, K, d = h64.shape
-    V, H = model.V, model.H
+    V = model.V
     if base is None:
         base = lm_head(h64, model.w_lm, model.dtype)
 
@@ -196,24 +225,10 @@ def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
     top2 = np.zeros((B, K))
     gap = np.zeros((B, K)) if forced is not None else None
     logits = np.zeros((B, K, V)) if want_logits else None
-
-    rid = np.arange(B) if request_ids is None else np.asarray(request_ids, dtype=np.int64)
-    s = np.zeros((B, H))
-    prev = np.asarray(anchor, dtype=np.int64).copy()
-    for p in range(K):                      # block position i = p + 1
-        x = model.embed_rows(prev)          # embedding of the token fed at this step
-        s = gru_cell(x, s, model.w_ih, model.w_hh, model.b_ih, model.b_hh)   # S_{i-1}
-        cat = np.concatenate([h64[:, p, :], s], axis=1)                      # [h_i ; S_{i-1}]
-        u = silu(cat @ model.w1.T)                                           # rank-r bottleneck
-        L = base[:, p, :] + u @ model.w2.T                                   # L_i = L_i^base + dL_i
+    for p, L, score, pick in positions(model, h64, anchor, base, mode=mode, temperature=temperature, seed=seed,
+                                       forced=forced, request_ids=request_ids):
         if logits is not None:
             logits[:, p, :] = L
-        if mode == "greedy":
-            score = L
-        else:
-            g = np.stack([gumbel_noise(seed, int(rid[b]), p + 1, V) for b in range(B)])
-            score = L / temperature + g
-        pick = np.argmax(score, axis=1)      # first index among equal maxima
         tokens[:, p] = pick
         srt = np.partition(score, V - 2, axis=1)[:, V - 2:]
         top2[:, p] = srt[:, 0]
@@ -221,8 +236,5 @@ def draft_block(model: Model, hidden: np.ndarray, anchor: np.ndarray, *,
         if forced is not None:
             fed = np.asarray(forced, dtype=np.int64)[:, p]
             gap[:, p] = top1[:, p] - score[np.arange(B), fed]
-            prev = fed
-        else:
-            prev = pick.astype(np.int64)
     tau = verify(tokens, target) if target is not None else None
     return Result(tokens, logits, base, top1, top2, gap, tau)

@@ -158,23 +158,24 @@ def make_weights(cfg: Config) -> Weights:
     return Weights(dt, w_lm, embed, w_ih, w_hh, b_ih, b_hh, w1, w2)
 
 
-def make_hidden(cfg: Config, B: int | None = None) -> np.ndarray:
+def make_hidden(cfg: Config, B: int | None = None, first: int = 0) -> np.ndarray:
     """Backbone hidden states [B, K, d] ~ N(0, 1) in storage form.
 
-    Requests are drawn independently, so the first B rows of a larger draw equal
-    a smaller draw (the batch sweep takes prefixes of one B=256 draw).
+    Request b is drawn from its own stream, so any slice of requests (the first B
+    of the batch sweep, one replica's share) matches the same rows of a larger
+    draw.  ``first`` is the global index of the first request returned.
     """
     B = cfg.B if B is None else B
-    rows = [_normal(cfg.seed, TID_HIDDEN * 1000003 + b, cfg.K * cfg.d, 1.0, cfg.dtype) for b in range(B)]
+    rows = [_normal(cfg.seed, TID_HIDDEN * 1000003 + first + b, cfg.K * cfg.d, 1.0, cfg.dtype) for b in range(B)]
     return np.stack(rows).reshape(B, cfg.K, cfg.d)
 
 
-def make_anchor(cfg: Config, B: int | None = None) -> np.ndarray:
+def make_anchor(cfg: Config, B: int | None = None, first: int = 0) -> np.ndarray:
     """Anchor (last confirmed) tokens [B] uniform in [0, V), int32."""
     B = cfg.B if B is None else B
     out = np.empty(B, dtype=np.int32)
     for b in range(B):
-        out[b] = np.random.default_rng([cfg.seed, TID_ANCHOR, b]).integers(0, cfg.V)
+        out[b] = np.random.default_rng([cfg.seed, TID_ANCHOR, first + b]).integers(0, cfg.V)
     return out
 
 
