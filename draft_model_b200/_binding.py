@@ -55,6 +55,7 @@ def load_library() -> ctypes.CDLL:
                                              ctypes.POINTER(ctypes.c_void_p)]),
         "domino_lm_head": (I32, [W, P, I32, I32, P, P, SZ, P]),
         "domino_correct_loop": (I32, [W, P, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
+        "domino_correct_loop_noalloc": (I32, [W, P, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P]),
         "domino_verify": (I32, [P, P, I32, I32, P, P]),
         "domino_draft_block_host": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, SZ, P]),
         "domino_poll": (I32, [P, P]),
@@ -182,6 +183,17 @@ def domino_correct_loop(w: DominoWeights, hidden, base, anchor, *, mode=0, tempe
                                               temperature, seed, _ptr(forced), _ptr(target), _ptr(draft_out),
                                               _ptr(logits_out), _ptr(tau_out), wp, wn, _stream(stream)),
            "domino_correct_loop")
+
+
+def domino_correct_loop_noalloc(w: DominoWeights, hidden, base, anchor, *, mode=0, temperature=1.0, seed=0,
+                                forced=None, target=None, draft_out, logits_out=None, tau_out=None,
+                                stream=None) -> None:
+    """Stage 2 without a workspace (scratch in a fixed array inside the library); waits for its work."""
+    B, K = draft_out.shape
+    _check(load_library().domino_correct_loop_noalloc(w.ref, _ptr(hidden), _ptr(base), _ptr(anchor), B, K, mode,
+                                                      temperature, seed, _ptr(forced), _ptr(target),
+                                                      _ptr(draft_out), _ptr(logits_out), _ptr(tau_out),
+                                                      _stream(stream)), "domino_correct_loop_noalloc")
 
 
 def domino_verify(draft, target, tau_out, stream=None) -> None:

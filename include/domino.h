@@ -146,6 +146,29 @@ DOMINO_API domino_status domino_correct_loop(const domino_weights* w, const void
                                   int32_t* tau_out, void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* Allocation-free variant of domino_correct_loop.  The pages have no
+ * counterpart: this exists for callers that cannot provide device memory —
+ * engines that reserve all device memory in their own arena and forbid other
+ * allocations, plugins running inside them, and deployments that must not
+ * allocate after start-up (cudaMalloc may synchronise the device and has no
+ * latency bound).  It takes no workspace and allocates nothing: its scratch is
+ * one fixed device array of 534,784 bytes inside the library, which every GPU
+ * that loads the library keeps until the process exits.  Arguments are those
+ * of domino_correct_loop without the workspace.
+ *   - Limits of that array: B <= 8, K <= 32, rank <= 256, gru_hidden <= 4096;
+ *     larger requests return DOMINO_ERR_UNSUPPORTED before any work.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - The call waits for its own work and returns what the device flagged
+ *     (DOMINO_OK, DOMINO_ERR_TIMEOUT or DOMINO_ERR_BAD_TOKEN).
+ *   - All calls share the array: calls whose work overlaps on one GPU (other
+ *     streams or host threads) race; run them one after another. */
+DOMINO_API domino_status domino_correct_loop_noalloc(const domino_weights* w, const void* hidden, const float* base,
+                                          const int32_t* anchor, int32_t B, int32_t K, int32_t mode,
+                                          float temperature, uint64_t seed, const int32_t* forced,
+                                          const int32_t* target, int32_t* draft_out, float* logits_out,
+                                          int32_t* tau_out, void* stream);
+
 /* Stage 3 only: tau_out[b] = number of leading i with draft[b, i] == target[b, i]. */
 DOMINO_API domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K,
                             int32_t* tau_out, void* stream);
