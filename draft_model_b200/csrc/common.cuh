@@ -53,14 +53,17 @@ __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
 }
 
 // Grid-wide barrier for a co-resident (cooperatively launched) grid, executed by
-// ONE thread per CTA (the caller brackets it with a CTA barrier).  The arrival
+// ONE thread per CTA (the caller brackets it with CTA barriers), in two halves
+// so a CTA can do independent work between arriving and waiting.  The arrival
 // counter only grows during a launch: barrier number k (0-based) completes when
 // it reaches G*(k+1).  Arrival is a fire-and-forget release reduction; the wait
 // polls with relaxed loads and ends with an acquire fence.  The last CTA to
 // leave the kernel resets the counter (grid_exit), so every launch starts at 0.
-// Returns false if the wait ran out of budget (the error bit is raised).
-__device__ __forceinline__ bool grid_barrier_one_thread(Control* ctl, uint32_t target, uint64_t budget_ns) {
+__device__ __forceinline__ void grid_barrier_arrive(Control* ctl) {
   asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&ctl->bar_count) : "memory");
+}
+// Returns false if the wait ran out of budget (the error bit is raised).
+__device__ __forceinline__ bool grid_barrier_wait(Control* ctl, uint32_t target, uint64_t budget_ns) {
   uint32_t spins = 0;
   uint64_t t0 = 0;
   while (true) {

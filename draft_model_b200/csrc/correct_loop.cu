@@ -11,22 +11,30 @@
 // and finally tau = leading agreement of t with the target tokens.
 //
 // B200 mapping.  One CTA per SM (148), all co-resident.  Each CTA statically owns
-//   * GRU hidden units [j0, j1): the three gate rows of W_ih and W_hh,
-//   * bottleneck rows [k0, k1) of W1,
+//   * GRU hidden units [j0, j1): the three gate rows of W_ih and W_hh and the
+//     matching columns of W1's state block (kept in shared memory),
+//   * bottleneck rows [k0, k1) (their W1_h h_i terms come from stage 1),
 //   * a contiguous vocabulary range [v0, v1) of W2 (balanced so every CTA streams
 //     about the same number of weight bytes per step).
 // A producer warp streams exactly those weight bytes, step after step, through a
-// shared-memory ring with 1-D bulk copies (TMA engine, no tensor map), and
-// issues bulk L2 prefetches a fixed distance ahead of the ring.  The weights
-// never depend on data, so HBM keeps streaming while consumers wait on grid
-// barriers.  Four consumer warps compute from the ring; item n is always handled
-// by warp n % 4 and lands in slot n % NSLOT (NSLOT a multiple of 4), so a slot is
-// only ever waited on by the warp that consumed its previous occupant.
-// Per step three bounded grid barriers: after the GRU (S_i complete), after the
-// bottleneck (u complete), after the vocabulary pass (argmax keys merged with a
-// 64-bit atomicMax).  W1 [h_i ; S] is split as W1_h h_i + W1_s S; the W1_h h_i
-// terms come precomputed from stage 1.  The CTA's slice of the base logits for
-// step i is copied into shared memory with cp.async while the GRU runs.
+// shared-memory ring with 1-D bulk copies (TMA engine, no tensor map) and bulk
+// L2 prefetches a fixed distance ahead of the ring.  The weights never depend on
+// data, so HBM keeps streaming while consumers wait on grid barriers.  Consumer
+// warps compute from the ring; item n is always handled by warp n % NCW and lands
+// in slot n % NSLOT (NSLOT a multiple of NCW), so a slot is only ever waited on
+// by the warp that consumed its previous occupant.
+//
+// Per step i, with two grid barriers:
+//   A  W_ih x_i partial dots (ring) -> GRU epilogue for own units (the W_hh S
+//      half was computed at the end of step i-1) -> each CTA's share of
+//      W1 [h_i ; S] (own state columns + own rows' h terms) added into a
+//      fixed-point int64 accumulator with red.add (exact, so order-free and
+//      deterministic)
+//   ---- barrier: S_i and the bottleneck pre-activation complete
+//   C  u = SiLU(acc); W2 row chunks (ring) + base logits (staged in shared memory
+//      with cp.async during A) -> per-lane argmax -> 64-bit atomicMax per request
+//   ---- barrier arrive; meanwhile W_hh S_i partial dots for step i+1 (ring);
+//        barrier wait -> picks, next embedding rows
 // Delta L and L_i never touch HBM unless final logits are requested.
 #include <cstdint>
 
@@ -37,12 +45,16 @@ namespace domino {
 
 namespace {
 
-constexpr int NCW = 4;                       // consumer warps
-constexpr int NTHREADS = (NCW + 1) * 32;     // + one producer warp
-constexpr int CONS_THREADS = NCW * 32;
 constexpr uint32_t BAR_CONS = 1;             // named barrier id among consumer warps
 constexpr int L2_AHEAD = 16;                 // items prefetched into L2 ahead of the ring
 constexpr int VCHUNK = 32;                   // W2 rows per ring item
+constexpr float kFixScale = 4294967296.0f;   // 2^32: fixed-point scale of the bottleneck accumulator
+
+// Consumer warps per CTA for a request group of NB: enough warps per scheduler to
+// hide FMA / shuffle / shared-memory latency, within the register file and the
+// shared memory left beside the larger groups' per-request state.
+template <int NB> struct Warps { static constexpr int NCW = NB <= 2 ? 12 : (NB == 4 ? 8 : 4); };
+constexpr int ncw_of(int NB) { return NB <= 2 ? 12 : (NB == 4 ? 8 : 4); }
 
 struct Partition {
   int j0, j1;  // GRU units
@@ -50,15 +62,16 @@ struct Partition {
   int v0, v1;  // vocabulary rows of W2
 };
 
-__device__ __host__ __forceinline__ long long vend_raw(const LoopArgs& a, int c, int G) {
+// Byte-balanced cut point of the vocabulary after CTA c (raw, before the
+// running maximum that makes the split monotone).
+__host__ __forceinline__ long long vend_raw(const LoopArgs& a, int c, int G) {
   if (c < 0) return 0;
   if (c >= G - 1) return a.V;
   const long long unitB = 3ll * (a.E + a.H) * a.wbytes;
-  const long long w1B = 1ll * a.H * a.wbytes;
   const long long rowB = 1ll * a.r * a.wbytes;
-  const long long total = 1ll * a.H * unitB + 1ll * a.r * w1B + 1ll * a.V * rowB;
+  const long long total = 1ll * a.H * unitB + 1ll * a.V * rowB;
   const long long target = total * (c + 1) / G;
-  const long long used = 1ll * ((c + 1) * a.H / G) * unitB + 1ll * ((c + 1) * a.r / G) * w1B;
+  const long long used = 1ll * ((c + 1) * a.H / G) * unitB;
   long long v = (target - used) / rowB;
   if (v < 0) v = 0;
   if (v > a.V) v = a.V;
@@ -94,14 +107,18 @@ struct Shared {
   float* S;        // [NB][H]   S_{i-1} (whole vector, all requests)
   uint8_t* x;      // [NB][E]   embedding of the fed token, storage type
   float* base;     // [NB][vmax] this CTA's slice of the step's base logits
-  float* part;     // [max_part][32] per-item partial sums
+  float* part_ih;  // [max_ih][32] partial sums of the W_ih items
+  float* part_hh;  // [max_hh][32] partial sums of the W_hh items
   float* hp;       // [kmax][NB][K] W1_h h terms of this CTA's rows
   float* bias;     // [umax][6] b_ih r,z,n then b_hh r,z,n of this CTA's units
+  float* w1s;      // [umax][r] W1 state-block columns of this CTA's units
+  float* s_own;    // [umax][NB] new state of this CTA's units
+  float* u;        // [NB][r] bottleneck output u = SiLU(W1 [h_i ; S_{i-1}])
   int* tok;        // [NB][K] picks (CTA 0 verifies from here)
   uint64_t* wbest; // [NCW][NB]
   int* flags;      // [0] abort
   int* fed;        // [NB] token fed to the GRU at the next step
-  uint8_t* items;  // [max_items] per-step ring item table (producer)
+  uint8_t* items;  // [per_step] ring item table (producer)
 };
 
 __device__ __forceinline__ Shared carve(uint8_t* base, const LoopArgs& a) {
@@ -112,9 +129,13 @@ __device__ __forceinline__ Shared carve(uint8_t* base, const LoopArgs& a) {
   s.S = reinterpret_cast<float*>(base + a.off_S);
   s.x = base + a.off_x;
   s.base = reinterpret_cast<float*>(base + a.off_base);
-  s.part = reinterpret_cast<float*>(base + a.off_part);
+  s.part_ih = reinterpret_cast<float*>(base + a.off_part);
+  s.part_hh = s.part_ih + static_cast<size_t>(a.max_ih) * 32;
   s.hp = reinterpret_cast<float*>(base + a.off_hp);
   s.bias = reinterpret_cast<float*>(base + a.off_bias);
+  s.w1s = reinterpret_cast<float*>(base + a.off_w1s);
+  s.s_own = reinterpret_cast<float*>(base + a.off_sown);
+  s.u = reinterpret_cast<float*>(base + a.off_u);
   s.tok = reinterpret_cast<int*>(base + a.off_tok);
   s.wbest = reinterpret_cast<uint64_t*>(base + a.off_wbest);
   s.flags = reinterpret_cast<int*>(base + a.off_flags);
@@ -130,53 +151,57 @@ __device__ __forceinline__ void set_abort(const Shared& s) {
   *reinterpret_cast<volatile int*>(&s.flags[0]) = 1;
 }
 
-// Consumer-wide grid barrier number k: named barrier, one thread arrives and
-// waits, named barrier.  Keeps control flow uniform even after an abort.
-__device__ __forceinline__ void consumer_grid_sync(const LoopArgs& a, const Shared& s, uint32_t k) {
+// Split grid barrier number k for the consumer warps.  arrive: after every
+// consumer has finished its writes, one thread publishes the CTA's arrival.
+// wait: one thread polls until all CTAs arrived, then every consumer proceeds.
+// Control flow stays uniform after an abort (the waits are skipped).
+template <int CONS_THREADS>
+__device__ __forceinline__ void grid_arrive(const LoopArgs& a, const Shared& s) {
   named_barrier(BAR_CONS, CONS_THREADS);
+  if (threadIdx.x == 0 && !aborted(s)) grid_barrier_arrive(a.ctl);
+}
+template <int CONS_THREADS>
+__device__ __forceinline__ void grid_wait(const LoopArgs& a, const Shared& s, uint32_t k) {
   if (threadIdx.x == 0 && !aborted(s)) {
-    if (!grid_barrier_one_thread(a.ctl, gridDim.x * (k + 1), a.budget_ns)) set_abort(s);
+    if (!grid_barrier_wait(a.ctl, gridDim.x * (k + 1), a.budget_ns)) set_abort(s);
   }
   named_barrier(BAR_CONS, CONS_THREADS);
 }
 
 // ---------------------------------------------------------------- per-step item schedule
+// Step i's ring items: [W_ih triples of own units] [W2 chunks] [W_hh triples of
+// own units, for step i+1; absent in the last step].
 struct Sched {
   Partition p;
-  Seg e3, h3, h1;
-  int nA, nB, nC, per_step;
+  Seg e3, h3;
+  int nIH, nC, nHH, per_step;
 };
 __device__ __forceinline__ Sched make_sched(const LoopArgs& a, int c, int G) {
   Sched s;
   s.p = partition_of(a, c, G);
   s.e3 = Seg{a.nsegE3, a.segE3};
   s.h3 = Seg{a.nsegH3, a.segH3};
-  s.h1 = Seg{a.nsegH1, a.segH1};
-  s.nA = (s.p.j1 - s.p.j0) * (s.e3.n + s.h3.n);
-  s.nB = (s.p.k1 - s.p.k0) * s.h1.n;
+  s.nIH = (s.p.j1 - s.p.j0) * s.e3.n;
+  s.nHH = (s.p.j1 - s.p.j0) * s.h3.n;
   s.nC = (s.p.v1 - s.p.v0 + VCHUNK - 1) / VCHUNK;
-  s.per_step = s.nA + s.nB + s.nC;
+  s.per_step = s.nIH + s.nC + s.nHH;
   return s;
 }
 
-// Source ranges of ring item n: `ncopy` copies of `bytes` each (3 gate rows of
-// one unit, one W1 row segment, or one W2 row chunk).
+// Source ranges of per-step item q: `ncopy` copies of `bytes` each.
 struct Item {
   const uint8_t* src[3];
   uint32_t bytes;
   int ncopy;
 };
-__device__ __forceinline__ Item item_of(const LoopArgs& a, const Sched& sc, int n) {
+__device__ __forceinline__ Item item_of(const LoopArgs& a, const Sched& sc, int q) {
   Item it;
-  int q = n % sc.per_step;
   const int wb = a.wbytes;
-  if (q < sc.nA) {
-    const int per_unit = sc.e3.n + sc.h3.n;
-    const int j = sc.p.j0 + q / per_unit;
-    const int s_all = q % per_unit;
-    const bool hh = s_all >= sc.e3.n;
-    const int s = hh ? s_all - sc.e3.n : s_all;
+  if (q < sc.nIH || q >= sc.nIH + sc.nC) {
+    const bool hh = q >= sc.nIH;
+    const int qq = hh ? q - sc.nIH - sc.nC : q;
     const Seg sg = hh ? sc.h3 : sc.e3;
+    const int j = sc.p.j0 + qq / sg.n, s = qq % sg.n;
     const int ncol = hh ? a.H : a.E;
     const uint8_t* m = static_cast<const uint8_t*>(hh ? a.w_hh : a.w_ih);
     const int c0 = s * sg.len, len = seg_len(sg, ncol, s);
@@ -185,18 +210,7 @@ __device__ __forceinline__ Item item_of(const LoopArgs& a, const Sched& sc, int 
     for (int g = 0; g < 3; ++g) it.src[g] = m + ((static_cast<size_t>(g) * a.H + j) * ncol + c0) * wb;
     return it;
   }
-  q -= sc.nA;
-  if (q < sc.nB) {
-    const int k = sc.p.k0 + q / sc.h1.n, s = q % sc.h1.n;
-    const int c0 = s * sc.h1.len, len = seg_len(sc.h1, a.H, s);
-    it.bytes = static_cast<uint32_t>(len) * wb;
-    it.ncopy = 1;
-    it.src[0] = static_cast<const uint8_t*>(a.w1) + (static_cast<size_t>(k) * (a.d + a.H) + a.d + c0) * wb;
-    it.src[1] = it.src[2] = nullptr;
-    return it;
-  }
-  q -= sc.nB;
-  const int v = sc.p.v0 + q * VCHUNK;
+  const int v = sc.p.v0 + (q - sc.nIH) * VCHUNK;
   const int rows = min(VCHUNK, sc.p.v1 - v);
   it.bytes = static_cast<uint32_t>(rows) * a.r * wb;
   it.ncopy = 1;
@@ -205,26 +219,37 @@ __device__ __forceinline__ Item item_of(const LoopArgs& a, const Sched& sc, int 
   return it;
 }
 
+// Walks the item sequence: q over the step's table, W_hh items skipped in the last step.
+struct Cursor {
+  int step, q;
+  __device__ __forceinline__ void next(const Sched& sc, int K) {
+    ++q;
+    if (step == K - 1 && q == sc.nIH + sc.nC) q = sc.per_step;
+    if (q >= sc.per_step) {
+      q = 0;
+      ++step;
+    }
+  }
+};
+
 // ---------------------------------------------------------------- producer
-// The per-step item sequence is identical for every step, so the producer
-// decodes it once into shared memory and then only walks the table.
 __device__ void producer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
   if ((threadIdx.x & 31) != 0) return;
+  if (sc.per_step == 0) return;
   Item* table = reinterpret_cast<Item*>(sh.items);
   for (int q = 0; q < sc.per_step; ++q) table[q] = item_of(a, sc, q);
   const uint64_t pol = policy_evict_first();
   const int nslot = a.nslot;
-  const int total = a.K * sc.per_step;
+  Cursor cur{0, 0}, ahead{0, 0};
   // warm L2 with the first items
-  int ahead_q = 0;
-  for (int p = 0; p < L2_AHEAD && p < total; ++p) {
-    const Item& it = table[ahead_q];
+  for (int p = 0; p < L2_AHEAD && ahead.step < a.K; ++p) {
+    const Item& it = table[ahead.q];
     for (int c = 0; c < it.ncopy; ++c) bulk_prefetch_l2(it.src[c], it.bytes);
-    if (++ahead_q == sc.per_step) ahead_q = 0;
+    ahead.next(sc, a.K);
   }
-  int n = 0, q = 0, slot = 0;
+  int n = 0, slot = 0;
   uint32_t phase = 0;
-  for (; n < total; ++n) {
+  for (; cur.step < a.K; ++n, cur.next(sc, a.K)) {
     if (n >= nslot) {
       const uint64_t t0 = globaltimer_ns();
       bool ok = true;
@@ -239,16 +264,15 @@ __device__ void producer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       }
       if (!ok) break;
     }
-    if (n + L2_AHEAD < total) {
-      const Item& ah = table[ahead_q];
+    if (ahead.step < a.K) {
+      const Item& ah = table[ahead.q];
       for (int c = 0; c < ah.ncopy; ++c) bulk_prefetch_l2(ah.src[c], ah.bytes);
-      if (++ahead_q == sc.per_step) ahead_q = 0;
+      ahead.next(sc, a.K);
     }
-    const Item& it = table[q];
+    const Item& it = table[cur.q];
     uint8_t* dst = sh.ring + static_cast<size_t>(slot) * kLoopSlotBytes;
     mbar_arrive_expect_tx(&sh.full[slot], it.bytes * it.ncopy);
     for (int c = 0; c < it.ncopy; ++c) bulk_g2s(dst + c * it.bytes, it.src[c], it.bytes, &sh.full[slot], pol);
-    if (++q == sc.per_step) q = 0;
     if (++slot == nslot) { slot = 0; phase ^= 1u; }
   }
   // drain: every issued copy must land before the CTA may exit
@@ -264,11 +288,6 @@ __device__ void producer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
 }
 
 // ---------------------------------------------------------------- consumer helpers
-template <typename W>
-__device__ __forceinline__ void load_vec8(const uint8_t* base, int idx, float* out) {
-  widen8(reinterpret_cast<const W*>(base) + idx, out);
-}
-
 // wait for item n (bound to this warp); returns the slot pointer or null on abort
 __device__ __forceinline__ const uint8_t* consume_begin(const LoopArgs& a, const Shared& sh, int n) {
   if (aborted(sh)) return nullptr;
@@ -284,7 +303,37 @@ __device__ __forceinline__ void consume_end(const LoopArgs& a, const Shared& sh,
   if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.empty[n % a.nslot]);
 }
 
-template <typename W>
+// Eight storage elements loaded raw from shared memory, widened later (keeps
+// several rows' loads in flight before the arithmetic that consumes them).
+template <typename W> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const uint8_t* base, int idx) {
+    v = *reinterpret_cast<const uint4*>(base + static_cast<size_t>(idx) * 2);
+  }
+  __device__ __forceinline__ void widen(float* out) const {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      out[2 * k] = __uint_as_float(w[k] << 16);
+      out[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const uint8_t* base, int idx) {
+    const float4* p = reinterpret_cast<const float4*>(base + static_cast<size_t>(idx) * 4);
+    a = p[0];
+    b = p[1];
+  }
+  __device__ __forceinline__ void widen(float* out) const {
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  }
+};
+
+template <typename W, int CONS_THREADS>
 __device__ __forceinline__ void gather_rows(const LoopArgs& a, const Shared& sh, int nrows) {
   const W* embed = static_cast<const W*>(a.embed);
   const int xg = a.E / 8;  // 8-element groups per embedding row
@@ -300,31 +349,91 @@ __device__ __forceinline__ void gather_rows(const LoopArgs& a, const Shared& sh,
   }
 }
 
-template <typename W, int NB>
+// Three gate-row dot products of one ring item (3 rows x len columns starting at
+// column c0) against NB vectors: the fed embeddings (ih) or the state (hh).
+// Lane l ends with slot l of [gate][request] (the warp's reduce-scatter).
+template <typename W, int NB, bool HH>
+__device__ __forceinline__ float gate_triple(const LoopArgs& a, const Shared& sh, const uint8_t* slot, int c0,
+                                             int len) {
+  const int lane = threadIdx.x & 31;
+  float acc[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+  for (int g = lane; g < len / 8; g += 32) {
+    Raw8<W> r0, r1, r2;
+    r0.load(slot, g * 8);
+    r1.load(slot, len + g * 8);
+    r2.load(slot, 2 * len + g * 8);
+    float w0[8], w1v[8], w2v[8];
+    r0.widen(w0);
+    r1.widen(w1v);
+    r2.widen(w2v);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float xv[8];
+      if (HH) {
+        const float* sp = sh.S + b * a.H + c0 + g * 8;
+        const float4 p0 = *reinterpret_cast<const float4*>(sp);
+        const float4 p1 = *reinterpret_cast<const float4*>(sp + 4);
+        xv[0] = p0.x; xv[1] = p0.y; xv[2] = p0.z; xv[3] = p0.w;
+        xv[4] = p1.x; xv[5] = p1.y; xv[6] = p1.z; xv[7] = p1.w;
+      } else {
+        Raw8<W> rx;
+        rx.load(sh.x, b * a.E + c0 + g * 8);
+        rx.widen(xv);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        acc[0 * NB + b] = fmaf(w0[e], xv[e], acc[0 * NB + b]);
+        acc[1 * NB + b] = fmaf(w1v[e], xv[e], acc[1 * NB + b]);
+        acc[2 * NB + b] = fmaf(w2v[e], xv[e], acc[2 * NB + b]);
+      }
+    }
+  }
+  return warp_reduce_scatter32(acc);
+}
+
+__device__ __forceinline__ long long* uacc_at(const LoopArgs& a, int buf, int b, int k) {
+  return a.u_acc + ((static_cast<size_t>(buf) * 8 + b) * a.r + k) * kUaccStride;
+}
+
+template <typename W, int NB, int NCW>
 __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
+  constexpr int CONS_THREADS = NCW * 32;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const bool cta0 = blockIdx.x == 0;
+  const int G = gridDim.x;
   const int nb = a.nb;
   const int K = a.K;
   const int kmine = sc.p.k1 - sc.p.k0;
   const int umine = sc.p.j1 - sc.p.j0;
   const int vrows = sc.p.v1 - sc.p.v0;
+  const W* w1 = static_cast<const W*>(a.w1);
   uint32_t nbar = 0;
 
-  // ---- prologue: argmax keys, biases, precomputed W1_h h terms, S = 0, first GRU input
+  // ---- prologue: zero argmax keys and this CTA's share of both accumulators,
+  // stage biases, W1 state columns and W1_h h terms, S = 0, first GRU input
   if (cta0)
     for (int q = tid; q < K * NB; q += CONS_THREADS) a.best[q] = 0ull;
+  for (int q = blockIdx.x * CONS_THREADS + tid; q < 2 * NB * a.r; q += G * CONS_THREADS)
+    *uacc_at(a, q / (NB * a.r), (q / a.r) % NB, q % a.r) = 0ll;
   for (int q = tid; q < umine * 6; q += CONS_THREADS) {
     const int jl = q / 6, g = q % 6;
     const float* bsrc = g < 3 ? a.b_ih : a.b_hh;
     sh.bias[q] = bsrc ? bsrc[(g % 3) * a.H + sc.p.j0 + jl] : 0.f;
+  }
+  for (int q = tid; q < umine * a.r; q += CONS_THREADS) {
+    const int jl = q / a.r, k = q % a.r;
+    const W wv = w1[static_cast<size_t>(k) * (a.d + a.H) + a.d + sc.p.j0 + jl];
+    sh.w1s[jl * a.r + k] = static_cast<float>(wv);
   }
   for (int q = tid; q < kmine * nb * K; q += CONS_THREADS) {
     const int kl = q / (nb * K), rem = q % (nb * K), b = rem / K, p = rem % K;
     sh.hp[(kl * NB + b) * K + p] = a.hp[(static_cast<size_t>(b) * K + p) * a.r + sc.p.k0 + kl];
   }
   for (int q = tid; q < NB * a.H; q += CONS_THREADS) sh.S[q] = 0.f;
+  for (int q = tid; q < sc.nHH * 32; q += CONS_THREADS) sh.part_hh[q] = 0.f;   // W_hh S_0 = 0
   if (tid < NB) {
     int t = tid < nb ? a.anchor[tid] : 0;
     if (t < 0 || t >= a.V) {
@@ -334,12 +443,13 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     sh.fed[tid] = t;
   }
   named_barrier(BAR_CONS, CONS_THREADS);
-  gather_rows<W>(a, sh, NB);
-  named_barrier(BAR_CONS, CONS_THREADS);
+  gather_rows<W, CONS_THREADS>(a, sh, NB);
+  grid_arrive<CONS_THREADS>(a, sh);         // zeroed keys and accumulators visible to all
+  grid_wait<CONS_THREADS>(a, sh, nbar++);
 
-  int n_base = 0;  // global item index of the first item of the current phase
-
+  int n = 0;  // global ring item index of the next item
   for (int i = 0; i < K; ++i) {
+    const int buf = i & 1;
     // base-logit slice of this step -> shared memory, overlapped with the GRU
     if (!aborted(sh)) {
       for (int q = tid; q < nb * vrows; q += CONS_THREADS) {
@@ -349,59 +459,24 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     }
     cp_async_commit();
 
-    // ================= phase A: GRU partial dot products
-    for (int q = 0; q < sc.nA; ++q) {
-      const int n = n_base + q;
-      if (n % NCW != warp) continue;
-      const uint8_t* slot = consume_begin(a, sh, n);
+    // ================= A: W_ih x partial dots
+    for (int q = 0; q < sc.nIH; ++q) {
+      const int nn = n + q;
+      if (nn % NCW != warp) continue;
+      const uint8_t* slot = consume_begin(a, sh, nn);
       if (slot) {
-        const int per_unit = sc.e3.n + sc.h3.n;
-        const int s_all = q % per_unit;
-        const bool side_hh = s_all >= sc.e3.n;
-        const int s = side_hh ? s_all - sc.e3.n : s_all;
-        const Seg sg = side_hh ? sc.h3 : sc.e3;
-        const int ncol = side_hh ? a.H : a.E;
-        const int c0 = s * sg.len, len = seg_len(sg, ncol, s);
-        float acc[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) acc[t] = 0.f;
-        for (int g = lane; g < len / 8; g += 32) {
-          float w0[8], w1v[8], w2v[8];
-          load_vec8<W>(slot, g * 8, w0);
-          load_vec8<W>(slot, len + g * 8, w1v);
-          load_vec8<W>(slot, 2 * len + g * 8, w2v);
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            float xv[8];
-            if (side_hh) {
-              const float* sp = sh.S + b * a.H + c0 + g * 8;
-              const float4 p0 = *reinterpret_cast<const float4*>(sp);
-              const float4 p1 = *reinterpret_cast<const float4*>(sp + 4);
-              xv[0] = p0.x; xv[1] = p0.y; xv[2] = p0.z; xv[3] = p0.w;
-              xv[4] = p1.x; xv[5] = p1.y; xv[6] = p1.z; xv[7] = p1.w;
-            } else {
-              load_vec8<W>(sh.x, b * a.E + c0 + g * 8, xv);
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              acc[0 * NB + b] = fmaf(w0[e], xv[e], acc[0 * NB + b]);
-              acc[1 * NB + b] = fmaf(w1v[e], xv[e], acc[1 * NB + b]);
-              acc[2 * NB + b] = fmaf(w2v[e], xv[e], acc[2 * NB + b]);
-            }
-          }
-        }
-        const float tot = warp_reduce_scatter32(acc);
-        sh.part[q * 32 + lane] = tot;
+        const int s = q % sc.e3.n;
+        const float tot = gate_triple<W, NB, false>(a, sh, slot, s * sc.e3.len, seg_len(sc.e3, a.E, s));
+        sh.part_ih[q * 32 + lane] = tot;
       }
-      consume_end(a, sh, n);
+      consume_end(a, sh, nn);
     }
-    n_base += sc.nA;
+    n += sc.nIH;
     named_barrier(BAR_CONS, CONS_THREADS);
 
     // GRU epilogue for own units: S_i[b][j]
     float* S_new = a.S_glob + static_cast<size_t>((i + 1) & 1) * NB * a.H;
     if (!aborted(sh)) {
-      const int per_unit = sc.e3.n + sc.h3.n;
       for (int q = tid; q < umine * NB; q += CONS_THREADS) {
         const int jl = q / NB, b = q % NB;
         const int j = sc.p.j0 + jl;
@@ -411,96 +486,77 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
           gh[g] = sh.bias[jl * 6 + 3 + g];
         }
         for (int s = 0; s < sc.e3.n; ++s)
-          for (int g = 0; g < 3; ++g) gi[g] += sh.part[(jl * per_unit + s) * 32 + g * NB + b];
+          for (int g = 0; g < 3; ++g) gi[g] += sh.part_ih[(jl * sc.e3.n + s) * 32 + g * NB + b];
         for (int s = 0; s < sc.h3.n; ++s)
-          for (int g = 0; g < 3; ++g) gh[g] += sh.part[(jl * per_unit + sc.e3.n + s) * 32 + g * NB + b];
+          for (int g = 0; g < 3; ++g) gh[g] += sh.part_hh[(jl * sc.h3.n + s) * 32 + g * NB + b];
         const float r = 1.f / (1.f + expf(-(gi[0] + gh[0])));
         const float z = 1.f / (1.f + expf(-(gi[1] + gh[1])));
         const float nn = tanhf(gi[2] + r * gh[2]);
         const float s_old = sh.S[b * a.H + j];
-        S_new[b * a.H + j] = (1.f - z) * nn + z * s_old;
+        const float s_new = (1.f - z) * nn + z * s_old;
+        S_new[b * a.H + j] = s_new;
+        sh.s_own[jl * NB + b] = s_new;
       }
     }
-    consumer_grid_sync(a, sh, nbar++);  // ---- barrier 1: S_i complete
+    named_barrier(BAR_CONS, CONS_THREADS);
+    // this CTA's share of the bottleneck pre-activation, in 2^-32 fixed point
+    if (!aborted(sh)) {
+      for (int q = tid; q < a.r * nb; q += CONS_THREADS) {
+        const int k = q % a.r, b = q / a.r;
+        const bool own_row = k >= sc.p.k0 && k < sc.p.k1;
+        if (umine == 0 && !own_row) continue;
+        float p = 0.f;
+        for (int jl = 0; jl < umine; ++jl) p = fmaf(sh.w1s[jl * a.r + k], sh.s_own[jl * NB + b], p);
+        if (own_row) p += sh.hp[((k - sc.p.k0) * NB + b) * K + i];
+        const long long fx = __float2ll_rn(p * kFixScale);
+        asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(uacc_at(a, buf, b, k)), "l"(fx) : "memory");
+      }
+    }
+    grid_arrive<CONS_THREADS>(a, sh);
+    grid_wait<CONS_THREADS>(a, sh, nbar++);   // ---- S_i and the pre-activation complete
 
-    // S_i -> shared (L1 bypassed: other SMs wrote it)
+    // S_i -> shared (L1 bypassed: other SMs wrote it); clear this CTA's share of
+    // the other accumulator for step i+1 (all reads of it ended before this barrier)
     if (!aborted(sh)) {
       for (int q = tid; q < NB * a.H / 4; q += CONS_THREADS)
         reinterpret_cast<float4*>(sh.S)[q] = __ldcg(reinterpret_cast<const float4*>(S_new) + q);
+      for (int q = blockIdx.x * CONS_THREADS + tid; q < NB * a.r; q += G * CONS_THREADS)
+        *uacc_at(a, buf ^ 1, q / a.r, q % a.r) = 0ll;
     }
-    named_barrier(BAR_CONS, CONS_THREADS);
-
-    // ================= phase B: u rows of this CTA
-    for (int q = 0; q < sc.nB; ++q) {
-      const int n = n_base + q;
-      if (n % NCW != warp) continue;
-      const uint8_t* slot = consume_begin(a, sh, n);
-      if (slot) {
-        const int s = q % sc.h1.n;
-        const int c0 = s * sc.h1.len, len = seg_len(sc.h1, a.H, s);
-        float acc[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) acc[t] = 0.f;
-        for (int g = lane; g < len / 8; g += 32) {
-          float wv[8];
-          load_vec8<W>(slot, g * 8, wv);
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const float* sp = sh.S + b * a.H + c0 + g * 8;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[b] = fmaf(wv[e], sp[e], acc[b]);
-          }
-        }
-        const float tot = warp_reduce_scatter32(acc);
-        sh.part[q * 32 + lane] = tot;
-      }
-      consume_end(a, sh, n);
-    }
-    n_base += sc.nB;
-    named_barrier(BAR_CONS, CONS_THREADS);
+    // u = SiLU(pre-activation): read once per CTA (one thread per entry) into
+    // shared memory, then every warp takes its registers from there
     if (!aborted(sh)) {
-      for (int q = tid; q < kmine * nb; q += CONS_THREADS) {
-        const int kl = q / nb, b = q % nb;
-        float pre = sh.hp[(kl * NB + b) * K + i];
-        for (int s = 0; s < sc.h1.n; ++s) pre += sh.part[(kl * sc.h1.n + s) * 32 + b];
-        const float silu = pre / (1.f + expf(-pre));
-        a.u_glob[b * a.r + sc.p.k0 + kl] = silu;
-      }
-    }
-    consumer_grid_sync(a, sh, nbar++);  // ---- barrier 2: u complete
-
-    // u -> registers: lane holds u[b][8*lane .. 8*lane+8)
-    float ureg[NB][8];
-#pragma unroll
-    for (int b = 0; b < NB; ++b)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ureg[b][e] = 0.f;
-    if (!aborted(sh) && lane * 8 < a.r) {
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        if (b < nb) {
-          const float4 p0 = __ldcg(reinterpret_cast<const float4*>(a.u_glob + b * a.r + lane * 8));
-          const float4 p1 = __ldcg(reinterpret_cast<const float4*>(a.u_glob + b * a.r + lane * 8 + 4));
-          ureg[b][0] = p0.x; ureg[b][1] = p0.y; ureg[b][2] = p0.z; ureg[b][3] = p0.w;
-          ureg[b][4] = p1.x; ureg[b][5] = p1.y; ureg[b][6] = p1.z; ureg[b][7] = p1.w;
-        }
+      for (int q = tid; q < nb * a.r; q += CONS_THREADS) {
+        const int b = q / a.r, k = q % a.r;
+        const long long fx = __ldcg(uacc_at(a, buf, b, k));
+        const float pre = static_cast<float>(static_cast<double>(fx) * (1.0 / 4294967296.0));
+        sh.u[b * a.r + k] = pre / (1.f + expf(-pre));
       }
     }
     cp_async_wait_all();
     named_barrier(BAR_CONS, CONS_THREADS);
+    float ureg[NB][8];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const bool have = b < nb && lane * 8 < a.r;
+      const float4 p0 = have ? *reinterpret_cast<const float4*>(sh.u + b * a.r + lane * 8) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 p1 = have ? *reinterpret_cast<const float4*>(sh.u + b * a.r + lane * 8 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      ureg[b][0] = p0.x; ureg[b][1] = p0.y; ureg[b][2] = p0.z; ureg[b][3] = p0.w;
+      ureg[b][4] = p1.x; ureg[b][5] = p1.y; ureg[b][6] = p1.z; ureg[b][7] = p1.w;
+    }
 
-    // ================= phase C: W2 chunks, residual, pick
+    // ================= C: W2 chunks, residual, pick
     constexpr int RPI = 32 / NB;           // rows per reduce-scatter round
     const int my_b = lane % NB;            // request whose sums this lane ends up with
     float best_s = -INFINITY;
     int best_v = 0x7FFFFFFF;
     const bool greedy = a.mode == 0;
     for (int q = 0; q < sc.nC; ++q) {
-      const int n = n_base + q;
-      if (n % NCW != warp) continue;
+      const int nn = n + q;
+      if (nn % NCW != warp) continue;
       const int vl0 = q * VCHUNK;          // chunk start, relative to v0
       const int rows = min(VCHUNK, vrows - vl0);
-      const uint8_t* slot = consume_begin(a, sh, n);
+      const uint8_t* slot = consume_begin(a, sh, nn);
       if (slot) {
 #pragma unroll
         for (int it = 0; it < NB; ++it) {
@@ -508,12 +564,21 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
 #pragma unroll
           for (int t = 0; t < 32; ++t) acc[t] = 0.f;
           if (lane * 8 < a.r) {
+            constexpr int BATCH = RPI < 8 ? RPI : 8;
 #pragma unroll
-            for (int rho = 0; rho < RPI; ++rho) {
-              const int rl = it * RPI + rho;
-              if (rl < rows) {
+            for (int rb = 0; rb < RPI; rb += BATCH) {
+              Raw8<W> raw[BATCH];
+#pragma unroll
+              for (int q2 = 0; q2 < BATCH; ++q2) raw[q2].load(slot, (it * RPI + rb + q2) * a.r + lane * 8);
+#pragma unroll
+              for (int q2 = 0; q2 < BATCH; ++q2) {
+                const int rho = rb + q2;
+                // rows past the chunk end read stale slot bytes: replace them by zero
+                const bool keep = (it * RPI + rho) < rows;
                 float wv[8];
-                load_vec8<W>(slot, rl * a.r + lane * 8, wv);
+                raw[q2].widen(wv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) wv[e] = keep ? wv[e] : 0.f;
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
@@ -533,9 +598,9 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
           }
         }
       }
-      consume_end(a, sh, n);
+      consume_end(a, sh, nn);
     }
-    n_base += sc.nC;
+    n += sc.nC;
     // merge lanes that hold the same request, then warps, then CTAs
 #pragma unroll
     for (int off = 16; off >= NB; off >>= 1) {
@@ -550,7 +615,24 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       for (int w = 0; w < NCW; ++w) k = max(k, sh.wbest[w * NB + tid]);
       if (k != 0ull) atomicMax(reinterpret_cast<unsigned long long*>(&a.best[i * NB + tid]), static_cast<unsigned long long>(k));
     }
-    consumer_grid_sync(a, sh, nbar++);  // ---- barrier 3: picks merged
+    grid_arrive<CONS_THREADS>(a, sh);
+
+    // ================= W_hh S_i partial dots for step i+1, overlapping the barrier
+    if (i + 1 < K) {
+      for (int q = 0; q < sc.nHH; ++q) {
+        const int nn = n + q;
+        if (nn % NCW != warp) continue;
+        const uint8_t* slot = consume_begin(a, sh, nn);
+        if (slot) {
+          const int s = q % sc.h3.n;
+          const float tot = gate_triple<W, NB, true>(a, sh, slot, s * sc.h3.len, seg_len(sc.h3, a.H, s));
+          sh.part_hh[q * 32 + lane] = tot;
+        }
+        consume_end(a, sh, nn);
+      }
+      n += sc.nHH;
+    }
+    grid_wait<CONS_THREADS>(a, sh, nbar++);   // ---- picks merged
 
     // picks, next GRU input
     if (tid < nb) {
@@ -567,7 +649,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       sh.fed[b] = f;
     }
     named_barrier(BAR_CONS, CONS_THREADS);
-    if (i + 1 < K && !aborted(sh)) gather_rows<W>(a, sh, nb);
+    if (i + 1 < K && !aborted(sh)) gather_rows<W, CONS_THREADS>(a, sh, nb);
     named_barrier(BAR_CONS, CONS_THREADS);
   }
 
@@ -582,14 +664,16 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
   if (tid == 0) grid_exit(a.ctl, gridDim.x);
 }
 
-template <typename W, int NB>
-__global__ void __launch_bounds__(NTHREADS, 1) correct_loop_kernel(const LoopArgs a) {
+template <typename W, int NB, int NCW>
+__global__ void __launch_bounds__((NCW + 1) * 32, 1) correct_loop_kernel(const LoopArgs a) {
+  constexpr int CONS_THREADS = NCW * 32;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int G = gridDim.x;
   if (a.selftest) {
     // one barrier episode that can never complete: exercises the bounded wait
     if (threadIdx.x == 0) {
-      grid_barrier_one_thread(a.ctl, static_cast<uint32_t>(G) + 1u, a.budget_ns);
+      grid_barrier_arrive(a.ctl);
+      grid_barrier_wait(a.ctl, static_cast<uint32_t>(G) + 1u, a.budget_ns);
       grid_exit(a.ctl, G);
     }
     return;
@@ -608,13 +692,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) correct_loop_kernel(const LoopArg
   if (threadIdx.x >= CONS_THREADS) {
     producer(a, sh, sc);
   } else {
-    consumer<W, NB>(a, sh, sc);
+    consumer<W, NB, NCW>(a, sh, sc);
   }
 }
 
 template <typename W, int NB>
 cudaError_t launch_one(const LoopArgs& a, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = correct_loop_kernel<W, NB>;
+  constexpr int NCW = Warps<NB>::NCW;
+  constexpr int NTHREADS = (NCW + 1) * 32;
+  auto kern = correct_loop_kernel<W, NB, NCW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -627,10 +713,11 @@ cudaError_t launch_one(const LoopArgs& a, int grid, size_t smem, cudaStream_t st
 
 }  // namespace
 
-// Shared-memory layout and segment plan for a request group of NB requests.
+// Shared-memory layout, vocabulary split and segment plan for a request group of NB.
 size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap) {
   const int wb = a.wbytes;
-  // segments: triples of rows fit one slot; single rows fit one slot
+  const int NCW = ncw_of(NB);
+  // segments: a triple of gate rows fits one slot
   auto plan = [](int total, int maxlen, int& nseg, int& len) {
     maxlen = maxlen / 8 * 8;
     nseg = (total + maxlen - 1) / maxlen;
@@ -638,11 +725,10 @@ size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap) {
   };
   plan(a.E, kLoopSlotBytes / (3 * wb), a.nsegE3, a.segE3);
   plan(a.H, kLoopSlotBytes / (3 * wb), a.nsegH3, a.segH3);
-  plan(a.H, kLoopSlotBytes / wb, a.nsegH1, a.segH1);
   const int umax = (a.H + grid - 1) / grid;
   const int kmax = (a.r + grid - 1) / grid;
-  a.max_part = umax * (a.nsegE3 + a.nsegH3);
-  a.max_part = a.max_part > kmax * a.nsegH1 ? a.max_part : kmax * a.nsegH1;
+  a.max_ih = umax * a.nsegE3;
+  a.max_hh = umax * a.nsegH3;
   if (grid > kLoopMaxGrid) return 0;
   // vocabulary split: running maximum of the byte-balanced cut points
   long long lo = 0;
@@ -657,7 +743,7 @@ size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap) {
   for (int c = 0; c < grid; ++c) {
     const Partition p = partition_of(a, c, grid);
     vmax = vmax > p.v1 - p.v0 ? vmax : p.v1 - p.v0;
-    const int n = (p.j1 - p.j0) * (a.nsegE3 + a.nsegH3) + (p.k1 - p.k0) * a.nsegH1 + (p.v1 - p.v0 + VCHUNK - 1) / VCHUNK;
+    const int n = (p.j1 - p.j0) * (a.nsegE3 + a.nsegH3) + (p.v1 - p.v0 + VCHUNK - 1) / VCHUNK;
     items_max = items_max > n ? items_max : n;
   }
   a.vmax = (vmax + 3) / 4 * 4;
@@ -666,9 +752,12 @@ size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap) {
       {&a.off_S, static_cast<size_t>(NB) * a.H * 4, 16},
       {&a.off_x, static_cast<size_t>(NB) * a.E * wb, 16},
       {&a.off_base, static_cast<size_t>(NB) * a.vmax * 4, 16},
-      {&a.off_part, static_cast<size_t>(a.max_part) * 32 * 4, 16},
+      {&a.off_part, static_cast<size_t>(a.max_ih + a.max_hh) * 32 * 4, 16},
       {&a.off_hp, static_cast<size_t>(kmax) * NB * a.K * 4, 16},
       {&a.off_bias, static_cast<size_t>(umax) * 6 * 4, 16},
+      {&a.off_w1s, static_cast<size_t>(umax) * a.r * 4, 16},
+      {&a.off_sown, static_cast<size_t>(umax) * NB * 4, 16},
+      {&a.off_u, static_cast<size_t>(NB) * a.r * 4, 16},
       {&a.off_tok, static_cast<size_t>(NB) * a.K * 4, 16},
       {&a.off_wbest, static_cast<size_t>(NCW) * NB * 8, 8},
       {&a.off_flags, 64, 16},
@@ -678,8 +767,9 @@ size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap) {
   for (const Piece& p : pieces) fixed = (fixed + p.align - 1) / p.align * p.align + p.bytes;
   fixed += 1024;
   if (fixed >= smem_cap) return 0;
-  int nslot = static_cast<int>((smem_cap - fixed) / kLoopSlotBytes) / NCW * NCW;
+  int nslot = static_cast<int>((smem_cap - fixed) / kLoopSlotBytes);
   if (nslot > 16) nslot = 16;
+  nslot = nslot / NCW * NCW;
   if (nslot < NCW) return 0;
   a.nslot = nslot;
   size_t off = static_cast<size_t>(nslot) * kLoopSlotBytes;
@@ -717,6 +807,6 @@ cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaS
   }
 }
 
-int loop_threads() { return NTHREADS; }
+int loop_threads(int NB) { return (ncw_of(NB) + 1) * 32; }
 
 }  // namespace domino

@@ -62,7 +62,7 @@ Layout layout_of(const domino_weights* w, int B, int K) {
   L.base = o; o += align_up(static_cast<size_t>(B) * K * w->vocab * 4);
   L.hp = o; o += align_up(static_cast<size_t>(B) * K * w->rank * 4);
   L.S = o; o += align_up(2ull * 8 * w->gru_hidden * 4);
-  L.u = o; o += align_up(8ull * w->rank * 4);
+  L.u = o; o += align_up(domino::uacc_bytes(w->rank));
   L.best = o; o += align_up(static_cast<size_t>(K) * 8 * 8);
   L.end = o;
   L.h_hidden = o; o += align_up(static_cast<size_t>(B) * K * w->d_model * wb);
@@ -128,7 +128,7 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
   a.w2 = w->w2;
   a.ctl = reinterpret_cast<Control*>(ws + L.ctl);
   a.S_glob = reinterpret_cast<float*>(ws + L.S);
-  a.u_glob = reinterpret_cast<float*>(ws + L.u);
+  a.u_acc = reinterpret_cast<long long*>(ws + L.u);
   const float* hp = reinterpret_cast<const float*>(ws + L.hp);
   a.best = reinterpret_cast<unsigned long long*>(ws + L.best);
   a.seed = seed;

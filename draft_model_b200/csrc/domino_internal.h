@@ -13,6 +13,11 @@ struct Control;
 constexpr uint32_t kLoopSlotBytes = 16384;
 // Largest grid the correction loop is planned for (one CTA per SM).
 constexpr int kLoopMaxGrid = 192;
+// int64 words between consecutive entries of the bottleneck accumulator (each
+// entry in its own 32-byte sector, so concurrent reductions do not share one).
+constexpr int kUaccStride = 4;
+// Bytes of the bottleneck accumulator: 2 buffers x 8 requests x rank entries.
+constexpr size_t uacc_bytes(int rank) { return 2ull * 8 * rank * kUaccStride * 8; }
 
 // Launch arguments of the persistent correction-loop kernel (one request group).
 struct LoopArgs {
@@ -38,7 +43,7 @@ struct LoopArgs {
   // scratch
   Control* ctl;
   float* S_glob;                 // [2][NB][H]
-  float* u_glob;                 // [NB][r]
+  long long* u_acc;              // [2][8][r] x kUaccStride: W1 [h ; S] in 2^-32 fixed point
   unsigned long long* best;      // [K][NB]
   uint64_t seed;
   uint64_t budget_ns;
@@ -50,20 +55,21 @@ struct LoopArgs {
   int32_t wbytes;   // 2 (bf16) or 4 (f32)
   int32_t selftest; // 1: run only the unreachable-barrier self-test
   // segment plan
-  int32_t segE3, nsegE3, segH3, nsegH3, segH1, nsegH1;
-  int32_t max_part;
+  int32_t segE3, nsegE3, segH3, nsegH3;
+  int32_t max_ih, max_hh;  // ring items of W_ih / W_hh per CTA per step, at most
   int32_t nslot;
   int32_t vmax;     // largest vocabulary slice of any CTA (rounded up to 4)
   int32_t vsplit[kLoopMaxGrid + 1];  // CTA c owns W2 rows [vsplit[c], vsplit[c+1])
   // shared-memory carve-up (byte offsets)
-  uint32_t off_bars, off_S, off_x, off_base, off_part, off_hp, off_bias, off_tok, off_wbest, off_flags, off_items;
+  uint32_t off_bars, off_S, off_x, off_base, off_part, off_hp, off_bias, off_w1s, off_sown, off_u, off_tok, off_wbest,
+      off_flags, off_items;
 };
 
 // Fills the segment plan and shared-memory offsets; returns the dynamic shared
 // memory size, or 0 if the shapes do not fit.
 size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap);
 int loop_group_size(int B);
-int loop_threads();
+int loop_threads(int NB);
 cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaStream_t stream);
 
 // LM head (stage 1).

@@ -6,7 +6,7 @@
 // not allocate after initialisation because cudaMalloc may synchronise the
 // device and has no latency bound.  This entry point needs no workspace and
 // allocates nothing: its scratch (control block, W1_h h terms, GRU state,
-// bottleneck vector, argmax keys) lives in one file-scope device array of fixed
+// bottleneck accumulator, argmax keys) lives in one file-scope device array of fixed
 // size, which every GPU that loads the library holds until the process exits.
 //
 // In host code the array's name is only a host-side stand-in, so the device
@@ -32,9 +32,9 @@ constexpr int kMaxH = 4096;    // GRU state width
 constexpr size_t kCtlBytes = 256;
 constexpr size_t kHpBytes = static_cast<size_t>(kMaxB) * kMaxK * kMaxR * 4;   // W1_h h terms [B,K,r]
 constexpr size_t kSBytes = 2ull * 8 * kMaxH * 4;                               // GRU state [2][8][H]
-constexpr size_t kUBytes = 8ull * kMaxR * 4;                                   // u [8][r]
+constexpr size_t kUBytes = domino::uacc_bytes(kMaxR);                           // bottleneck accumulator
 constexpr size_t kBestBytes = static_cast<size_t>(kMaxK) * 8 * 8;              // argmax keys [K][8]
-constexpr size_t kScratchBytes = kCtlBytes + kHpBytes + kSBytes + kUBytes + kBestBytes;  // 534,784 bytes
+constexpr size_t kScratchBytes = kCtlBytes + kHpBytes + kSBytes + kUBytes + kBestBytes;  // 657,664 bytes
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -105,7 +105,7 @@ extern "C" domino_status domino_correct_loop_noalloc(const domino_weights* w, co
   domino::Control* ctl = reinterpret_cast<domino::Control*>(s);
   float* hp = reinterpret_cast<float*>(s + kCtlBytes);
   float* S = reinterpret_cast<float*>(s + kCtlBytes + kHpBytes);
-  float* u = reinterpret_cast<float*>(s + kCtlBytes + kHpBytes + kSBytes);
+  long long* uacc = reinterpret_cast<long long*>(s + kCtlBytes + kHpBytes + kSBytes);
   unsigned long long* best = reinterpret_cast<unsigned long long*>(s + kCtlBytes + kHpBytes + kSBytes + kUBytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -138,7 +138,7 @@ extern "C" domino_status domino_correct_loop_noalloc(const domino_weights* w, co
   a.w2 = w->w2;
   a.ctl = ctl;
   a.S_glob = S;
-  a.u_glob = u;
+  a.u_acc = uacc;
   a.best = best;
   a.seed = seed;
   a.budget_ns = kBudgetNs;

@@ -152,7 +152,7 @@ DOMINO_API domino_status domino_correct_loop(const domino_weights* w, const void
  * allocations, plugins running inside them, and deployments that must not
  * allocate after start-up (cudaMalloc may synchronise the device and has no
  * latency bound).  It takes no workspace and allocates nothing: its scratch is
- * one fixed device array of 534,784 bytes inside the library, which every GPU
+ * one fixed device array of 657,664 bytes inside the library, which every GPU
  * that loads the library keeps until the process exits.  Arguments are those
  * of domino_correct_loop without the workspace.
  *   - Limits of that array: B <= 8, K <= 32, rank <= 256, gru_hidden <= 4096;
