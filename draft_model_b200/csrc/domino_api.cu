@@ -29,8 +29,13 @@ int num_sms() {
   return n;
 }
 
+// The control region (zeroed by domino_workspace_init and after device errors)
+// holds the control block and the stream-K ready flags of the LM head.
+constexpr size_t kCtlRegion = 1024;
+static_assert(sizeof(Control) + domino::kLoopMaxGrid * 4 <= kCtlRegion, "control region");
+
 struct Layout {
-  size_t ctl, base, hp, S, u, best, end;                   // device workspace
+  size_t ctl, skflag, base, hp, S, u, best, skp, end;      // device workspace
   size_t h_hidden, h_anchor, h_forced, h_target, h_draft, h_tau, h_end;  // host-variant staging
 };
 
@@ -58,12 +63,15 @@ Layout layout_of(const domino_weights* w, int B, int K) {
   Layout L{};
   const size_t wb = w->dtype == DOMINO_BF16 ? 2 : 4;
   size_t o = 0;
-  L.ctl = o; o += align_up(sizeof(Control));
+  L.ctl = o;
+  L.skflag = o + sizeof(Control);
+  o += kCtlRegion;
   L.base = o; o += align_up(static_cast<size_t>(B) * K * w->vocab * 4);
   L.hp = o; o += align_up(static_cast<size_t>(B) * K * w->rank * 4);
   L.S = o; o += align_up(2ull * 8 * w->gru_hidden * 4);
   L.u = o; o += align_up(domino::uacc_bytes(w->rank));
   L.best = o; o += align_up(static_cast<size_t>(K) * 8 * 8);
+  L.skp = o; o += align_up(domino::lm_head_sk_bytes(B * K));
   L.end = o;
   L.h_hidden = o; o += align_up(static_cast<size_t>(B) * K * w->d_model * wb);
   L.h_anchor = o; o += align_up(static_cast<size_t>(B) * 4);
@@ -90,15 +98,17 @@ domino_status check_workspace(void* ws, size_t bytes, size_t need) {
 // Stage 1: base logits (base != null) and/or the hidden-state half of the
 // bottleneck pre-activation hp[m, k] = W1[k, 0:d] h[m] (hp != null).
 domino_status run_lm_head(const domino_weights* w, const void* hidden, int B, int K, float* base, float* hp,
-                          Control* ctl, cudaStream_t st) {
+                          char* ws, const Layout& L, cudaStream_t st) {
+  Control* ctl = reinterpret_cast<Control*>(ws + L.ctl);
   const int M = B * K;
   const int w1_stride = w->d_model + w->gru_hidden;
   cudaError_t e = cudaSuccess;
   if (w->dtype == DOMINO_BF16) {
     const int sms = num_sms();
     if (sms <= 0) return DOMINO_ERR_CUDA;
-    e = domino::launch_lm_head_tc(w->w_lm, hidden, base, w->vocab, M, w->d_model, w->w1, w->rank, w1_stride, hp, ctl,
-                                  g_budget_ns.load(), sms, st);
+    e = domino::launch_lm_head_tc(w->w_lm, hidden, base, w->vocab, M, w->d_model, w->w1, w->rank, w1_stride, hp,
+                                  reinterpret_cast<float*>(ws + L.skp), reinterpret_cast<uint32_t*>(ws + L.skflag),
+                                  ctl, g_budget_ns.load(), sms, st);
   } else {
     const float* h = static_cast<const float*>(hidden);
     if (base) e = domino::launch_lm_head_f32(static_cast<const float*>(w->w_lm), h, base, w->vocab, M, w->d_model,
@@ -196,9 +206,9 @@ size_t domino_workspace_bytes_host(const domino_weights* w, int32_t B, int32_t K
 }
 
 domino_status domino_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < sizeof(Control))
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < kCtlRegion)
     return DOMINO_ERR_WORKSPACE;
-  return from_cuda(cudaMemsetAsync(workspace, 0, sizeof(Control), static_cast<cudaStream_t>(stream)));
+  return from_cuda(cudaMemsetAsync(workspace, 0, kCtlRegion, static_cast<cudaStream_t>(stream)));
 }
 
 domino_status domino_lm_head(const domino_weights* w, const void* hidden, int32_t B, int32_t K, float* base_out,
@@ -206,9 +216,10 @@ domino_status domino_lm_head(const domino_weights* w, const void* hidden, int32_
   if (!weights_ok(w) || !weight_ptrs_ok(w, true, false)) return DOMINO_ERR_INVALID_ARG;
   if (B < 1 || K < 1 || K > 32 || !hidden || !aligned16(hidden) || !base_out || !aligned16(base_out))
     return DOMINO_ERR_INVALID_ARG;
-  const domino_status ws = check_workspace(workspace, workspace_bytes, sizeof(Control));
+  const Layout L = layout_of(w, B, K);
+  const domino_status ws = check_workspace(workspace, workspace_bytes, L.end);
   if (ws != DOMINO_OK) return ws;
-  return run_lm_head(w, hidden, B, K, base_out, nullptr, static_cast<Control*>(workspace),
+  return run_lm_head(w, hidden, B, K, base_out, nullptr, static_cast<char*>(workspace), L,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -226,8 +237,7 @@ domino_status domino_correct_loop(const domino_weights* w, const void* hidden, c
   if (s != DOMINO_OK) return s;
   char* ws = static_cast<char*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = run_lm_head(w, hidden, B, K, nullptr, reinterpret_cast<float*>(ws + L.hp), reinterpret_cast<Control*>(ws + L.ctl),
-                  st);
+  s = run_lm_head(w, hidden, B, K, nullptr, reinterpret_cast<float*>(ws + L.hp), ws, L, st);
   if (s != DOMINO_OK) return s;
   return run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out,
                   tau_out, ws, L, st);
@@ -253,8 +263,7 @@ domino_status domino_draft_block_events(const domino_weights* w, const void* hid
   };
   if ((s = mark(0)) != DOMINO_OK) return s;
   float* base = reinterpret_cast<float*>(ws + L.base);
-  s = run_lm_head(w, hidden, B, K, base, reinterpret_cast<float*>(ws + L.hp), reinterpret_cast<Control*>(ws + L.ctl),
-                  st);
+  s = run_lm_head(w, hidden, B, K, base, reinterpret_cast<float*>(ws + L.hp), ws, L, st);
   if (s != DOMINO_OK) return s;
   if ((s = mark(1)) != DOMINO_OK) return s;
   s = run_loop(w, hidden, base, anchor, B, K, mode, temperature, seed, forced, target, draft_out, logits_out, tau_out,
@@ -320,7 +329,7 @@ domino_status domino_poll(void* workspace, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return from_cuda(e);
   if (err == 0) return DOMINO_OK;
-  e = cudaMemsetAsync(workspace, 0, sizeof(Control), st);
+  e = cudaMemsetAsync(workspace, 0, kCtlRegion, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return from_cuda(e);
   if (err & domino::ERRBIT_TIMEOUT) return DOMINO_ERR_TIMEOUT;
@@ -330,7 +339,7 @@ domino_status domino_poll(void* workspace, void* stream) {
 void domino_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns ? ns : 1); }
 
 domino_status domino_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint64_t budget_ns, void* stream) {
-  const domino_status s = check_workspace(workspace, workspace_bytes, sizeof(Control));
+  const domino_status s = check_workspace(workspace, workspace_bytes, kCtlRegion);
   if (s != DOMINO_OK) return s;
   const int sms = num_sms();
   if (sms <= 0) return DOMINO_ERR_CUDA;

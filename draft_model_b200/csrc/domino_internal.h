@@ -75,9 +75,17 @@ cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaS
 // LM head (stage 1).
 // out [M, V] = hidden . W_lm^T (skipped if out is null); out2 [M, rows2] =
 // hidden . W1[:, 0:Kd]^T with W1 rows w1_stride elements apart (skipped if null).
+// sk_part / sk_flag: stream-K scratch (partial tiles [kLoopMaxGrid][BN][128] fp32
+// and [kLoopMaxGrid] flags, zero between launches), or null for whole tiles only.
 cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd,
-                              const void* w1, int rows2, int w1_stride, float* out2, Control* ctl,
-                              uint64_t budget_ns, int num_sms, cudaStream_t stream);
+                              const void* w1, int rows2, int w1_stride, float* out2, float* sk_part,
+                              uint32_t* sk_flag, Control* ctl, uint64_t budget_ns, int num_sms,
+                              cudaStream_t stream);
+// Bytes of stream-K partial tiles for M block positions.
+inline size_t lm_head_sk_bytes(int M) {
+  const int bn = ((M + 15) / 16 * 16) > 256 ? 256 : (M + 15) / 16 * 16;
+  return static_cast<size_t>(kLoopMaxGrid) * bn * 128 * 4;
+}
 cudaError_t launch_lm_head_f32(const float* w, const float* hidden, float* out, int V, int M, int Kd, int ldw,
                                cudaStream_t stream);
 

@@ -36,19 +36,64 @@ constexpr int BM = 128;        // vocabulary rows per tile (UMMA M)
 constexpr int BK = 64;         // bf16 elements per k-block (one 128-byte swizzle atom row)
 constexpr int NTH = 192;
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;  // 16 KB
+constexpr int kStageSubBlocks = 2;               // 64-wide k sub-blocks per pipeline stage
 
 struct TcArgs {
   float* out;        // [M, V]
   float* out2;       // [M, rows2] (second A operand's products) or null
+  float* sk_part;    // stream-K partial tiles [grid][BN][128] or null (whole tiles only)
+  uint32_t* sk_flag; // [grid] partial-tile ready flags (zero between launches)
   Control* ctl;
   uint64_t budget_ns;
   int V, M, Kd;
   int BN;            // block positions per tile (multiple of 16, <= 256)
+  int nk;            // 64-wide k sub-blocks per pipeline stage
   int stages;
   int tmem_cols;     // power of two >= 2*BN
-  int num_vt, num_mt, num_kb;
+  int num_vt, num_mt, num_kb;  // num_kb counts pipeline stages (nk sub-blocks each) per tile
   int rows2, num_vt2;  // second A operand: rows and 128-row tiles (0 = none)
 };
+
+// A contiguous run of k-stages of one tile handled by one CTA.  FULL runs cover
+// the whole tile; with stream-K a CTA's first run may be the TAIL of a tile
+// whose HEAD is the previous CTA's last run: the TAIL's owner parks its partial
+// sums in global memory and the HEAD's owner adds them and stores the tile.
+enum SegKind : int { SEG_FULL = 0, SEG_TAIL = 1, SEG_HEAD = 2 };
+struct Seg {
+  int t, kb0, kb1, kind;
+};
+struct SegIter {
+  long long u, hi;  // stream-K: unit range (units = k-stages over all tiles)
+  int t;            // whole-tile schedule: next tile
+  bool sk;
+  __device__ __forceinline__ bool next(const TcArgs& a, int ntiles, Seg& g) {
+    if (sk) {
+      if (u >= hi) return false;
+      g.t = static_cast<int>(u / a.num_kb);
+      g.kb0 = static_cast<int>(u % a.num_kb);
+      g.kb1 = static_cast<int>(min(static_cast<long long>(a.num_kb), g.kb0 + (hi - u)));
+      g.kind = (g.kb0 == 0 && g.kb1 == a.num_kb) ? SEG_FULL : (g.kb0 > 0 ? SEG_TAIL : SEG_HEAD);
+      u += g.kb1 - g.kb0;
+      return true;
+    }
+    if (t >= ntiles) return false;
+    g.t = t;
+    g.kb0 = 0;
+    g.kb1 = a.num_kb;
+    g.kind = SEG_FULL;
+    t += gridDim.x;
+    return true;
+  }
+};
+__device__ __forceinline__ SegIter seg_begin(const TcArgs& a, int ntiles) {
+  SegIter it;
+  it.sk = a.sk_part != nullptr;
+  const long long units = static_cast<long long>(ntiles) * a.num_kb;
+  it.u = units * blockIdx.x / gridDim.x;
+  it.hi = units * (blockIdx.x + 1) / gridDim.x;
+  it.t = blockIdx.x;
+  return it;
+}
 
 // ---- tcgen05 / TMA primitives (inline PTX) ----
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
@@ -118,8 +163,9 @@ __global__ void __launch_bounds__(NTH, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment of every stage (the swizzle atom)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t b_stage_bytes = static_cast<uint32_t>(a.BN) * BK * 2;
-  const uint32_t stage_bytes = A_STAGE_BYTES + b_stage_bytes;
+  const uint32_t b_sub_bytes = static_cast<uint32_t>(a.BN) * BK * 2;
+  const uint32_t a_bytes = A_STAGE_BYTES * a.nk;          // nk A sub-tiles, then nk B sub-tiles
+  const uint32_t stage_bytes = a_bytes + b_sub_bytes * a.nk;
   uint8_t* ctrl = smem + static_cast<size_t>(a.stages) * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* empty = full + a.stages;
@@ -173,21 +219,26 @@ __global__ void __launch_bounds__(NTH, 1)
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
-      int it = 0;  // global k-block counter
+      int it = 0;  // global k-stage counter
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const bool second = t < ntiles2;
-        const int tt = second ? t : t - ntiles2;
+      SegIter si = seg_begin(a, ntiles);
+      Seg g;
+      while (ok && si.next(a, ntiles, g)) {
+        const bool second = g.t < ntiles2;
+        const int tt = second ? g.t : g.t - ntiles2;
         const int vt = tt / a.num_mt, mt = tt % a.num_mt;
         const CUtensorMap* tA = second ? &tmA2 : &tmA;
-        for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+        for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
           const int s = it % a.stages;
           if (it >= a.stages && !bounded_wait(&empty[s], ((it / a.stages) - 1) & 1)) { ok = false; break; }
           uint8_t* sa = smem + static_cast<size_t>(s) * stage_bytes;
-          uint8_t* sb = sa + A_STAGE_BYTES;
+          uint8_t* sb = sa + a_bytes;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
-          tma_load_2d(sa, tA, kb * BK, vt * BM, &full[s]);
-          tma_load_2d(sb, &tmB, kb * BK, mt * a.BN, &full[s]);
+          for (int j = 0; j < a.nk; ++j) {
+            const int kc = (kb * a.nk + j) * BK;
+            tma_load_2d(sa + j * A_STAGE_BYTES, tA, kc, vt * BM, &full[s]);
+            tma_load_2d(sb + j * b_sub_bytes, &tmB, kc, mt * a.BN, &full[s]);
+          }
         }
       }
       // drain copies that were issued but may still be in flight
@@ -204,25 +255,31 @@ __global__ void __launch_bounds__(NTH, 1)
       const uint32_t idesc = idesc_bf16_f32(a.BN);
       int it = 0, local = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
+      SegIter si = seg_begin(a, ntiles);
+      Seg g;
+      while (ok && si.next(a, ntiles, g)) {
         const int acc = local & 1;
         if (local >= 2 && !bounded_wait(&tempty[acc], ((local >> 1) - 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
-        for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+        for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
           const int s = it % a.stages;
           if (!bounded_wait(&full[s], (it / a.stages) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-          const uint32_t sb = sa + A_STAGE_BYTES;
+          const uint32_t sb = sa + a_bytes;
+          for (int j = 0; j < a.nk; ++j) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            tc_mma_bf16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
-                        (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              tc_mma_bf16(d_tmem, smem_desc_sw128(sa + j * A_STAGE_BYTES + kk * 32),
+                          smem_desc_sw128(sb + j * b_sub_bytes + kk * 32), idesc,
+                          (kb > g.kb0 || j > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&empty[s]);   // frees the stage once these MMAs have read it
         }
         if (ok) tc_commit(&tfull[acc]);
+        ++local;
       }
       // every MMA issued by this thread must finish before TMEM is released
       tc_commit(mma_done);
@@ -235,32 +292,73 @@ __global__ void __launch_bounds__(NTH, 1)
     // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4
     const int q = warp & 3;
     int local = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+    SegIter si = seg_begin(a, ntiles);
+    Seg g;
+    while (si.next(a, ntiles, g)) {
       const int acc = local & 1;
-      bool ok = true;
-      if (lane == 0) ok = bounded_wait(&tfull[acc], (local >> 1) & 1);
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
+      if (lane == 0) bounded_wait(&tfull[acc], (local >> 1) & 1);
+      named_barrier(2, 128);          // the four epilogue warps take the same decision
+      if (*abort_flag) break;
       tc_fence_after();
-      const bool second = t < ntiles2;
-      const int tt = second ? t : t - ntiles2;
+      const bool second = g.t < ntiles2;
+      const int tt = second ? g.t : g.t - ntiles2;
       const int vt = tt / a.num_mt, mt = tt % a.num_mt;
-      const int v = vt * BM + q * 32 + lane;
+      const int row = q * 32 + lane;                 // row of the 128-row tile
+      const int v = vt * BM + row;
       const int nrows = second ? a.rows2 : a.V;
       float* dst = second ? a.out2 : a.out;
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      if (g.kind == SEG_HEAD) {
+        // the next CTA parked the tail of this tile: wait for its flag
+        bool ready = true;
+        if (threadIdx.x == 64) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_u32(&a.sk_flag[blockIdx.x + 1]) == 0u) {
+            if (*abort_flag || globaltimer_ns() - t0 > a.budget_ns) {
+              raise_error(a.ctl, ERRBIT_TIMEOUT);
+              *abort_flag = 1;
+              ready = false;
+              break;
+            }
+          }
+        }
+        named_barrier(2, 128);
+        ready = ready && !*abort_flag;
+        if (!ready) break;
+      }
+      const float* park_in = a.sk_part + static_cast<size_t>(blockIdx.x + 1) * a.BN * BM;
+      float* park_out = a.sk_part + static_cast<size_t>(blockIdx.x) * a.BN * BM;
       for (int c0 = 0; c0 < a.BN; c0 += 16) {
         float vals[16];
         tmem_ld16(trow + c0, vals);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const int m = mt * a.BN + c0 + c;
-          if (v < nrows && m < a.M) dst[static_cast<size_t>(m) * nrows + v] = vals[c];
+          const int col = c0 + c;
+          if (g.kind == SEG_TAIL) {
+            park_out[static_cast<size_t>(col) * BM + row] = vals[c];
+          } else {
+            float x = vals[c];
+            if (g.kind == SEG_HEAD) x += __ldcg(park_in + static_cast<size_t>(col) * BM + row);
+            const int m = mt * a.BN + col;
+            if (v < nrows && m < a.M) dst[static_cast<size_t>(m) * nrows + v] = x;
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (g.kind != SEG_FULL) {
+        named_barrier(2, 128);   // all four epilogue warps done with the partial tile
+        if (threadIdx.x == 64) {
+          if (g.kind == SEG_TAIL) {
+            __threadfence();
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&a.sk_flag[blockIdx.x]), "r"(1u) : "memory");
+          } else {
+            st_relaxed_u32(&a.sk_flag[blockIdx.x + 1], 0u);   // consumed: clean for the next launch
+          }
+        }
+      }
+      ++local;
     }
   }
   tc_fence_before();
@@ -302,8 +400,9 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, int rows, int cols, int box_row
 }  // namespace
 
 cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, int V, int M, int Kd,
-                              const void* w1, int rows2, int w1_stride, float* out2, Control* ctl, uint64_t budget_ns,
-                              int num_sms, cudaStream_t stream) {
+                              const void* w1, int rows2, int w1_stride, float* out2, float* sk_part,
+                              uint32_t* sk_flag, Control* ctl, uint64_t budget_ns, int num_sms,
+                              cudaStream_t stream) {
   TcArgs a;
   a.out = out;
   a.out2 = out2;
@@ -321,8 +420,9 @@ cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, 
   a.num_vt = out ? (V + BM - 1) / BM : 0;
   a.num_vt2 = out2 ? (rows2 + BM - 1) / BM : 0;
   a.num_mt = (M + a.BN - 1) / a.BN;
-  a.num_kb = (Kd + BK - 1) / BK;
-  const uint32_t stage_bytes = A_STAGE_BYTES + static_cast<uint32_t>(a.BN) * BK * 2;
+  a.nk = a.BN <= 64 ? kStageSubBlocks : 1;
+  a.num_kb = (Kd + BK * a.nk - 1) / (BK * a.nk);
+  const uint32_t stage_bytes = (A_STAGE_BYTES + static_cast<uint32_t>(a.BN) * BK * 2) * a.nk;
   const size_t budget = 220 * 1024;
   int stages = static_cast<int>((budget - 2048) / stage_bytes);
   if (stages > 12) stages = 12;
@@ -345,8 +445,15 @@ cudaError_t launch_lm_head_tc(const void* w_lm, const void* hidden, float* out, 
   const int ntiles = (a.num_vt + a.num_vt2) * a.num_mt;
   if (ntiles == 0) return cudaSuccess;
   const int grid = ntiles < num_sms ? ntiles : num_sms;
-  lm_head_tc_kernel<<<grid, NTH, smem, stream>>>(tmA, tmA2, tmB, a);
-  return cudaGetLastError();
+  // stream-K when whole tiles would leave a ragged last wave and every CTA still
+  // gets at least one tile's worth of k-stages (so a tile spans at most two CTAs)
+  const long long units = static_cast<long long>(ntiles) * a.num_kb;
+  const bool sk = sk_part && sk_flag && grid <= kLoopMaxGrid && ntiles % grid != 0 && units / grid >= a.num_kb;
+  a.sk_part = sk ? sk_part : nullptr;
+  a.sk_flag = sk ? sk_flag : nullptr;
+  void* params[] = {&tmA, &tmA2, &tmB, &a};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(lm_head_tc_kernel), dim3(grid), dim3(NTH), params, smem,
+                                     stream);
 }
 
 }  // namespace domino

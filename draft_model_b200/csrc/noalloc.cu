@@ -117,8 +117,8 @@ extern "C" domino_status domino_correct_loop_noalloc(const domino_weights* w, co
   const int M = B * K;
   const int w1_stride = w->d_model + w->gru_hidden;
   if (w->dtype == DOMINO_BF16)
-    e = domino::launch_lm_head_tc(nullptr, hidden, nullptr, w->vocab, M, w->d_model, w->w1, w->rank, w1_stride, hp, ctl,
-                                  kBudgetNs, sms, st);
+    e = domino::launch_lm_head_tc(nullptr, hidden, nullptr, w->vocab, M, w->d_model, w->w1, w->rank, w1_stride, hp,
+                                  nullptr, nullptr, ctl, kBudgetNs, sms, st);
   else
     e = domino::launch_lm_head_f32(static_cast<const float*>(w->w1), static_cast<const float*>(hidden), hp, w->rank, M,
                                    w->d_model, w1_stride, st);
