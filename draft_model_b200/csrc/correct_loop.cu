@@ -46,15 +46,21 @@ namespace domino {
 namespace {
 
 constexpr uint32_t BAR_CONS = 1;             // named barrier id among consumer warps
-constexpr int L2_AHEAD = 16;                 // items prefetched into L2 ahead of the ring
+constexpr int L2_AHEAD = 32;                 // items prefetched into L2 ahead of the ring's next item
 constexpr int VCHUNK = 32;                   // W2 rows per ring item
 constexpr float kFixScale = 4294967296.0f;   // 2^32: fixed-point scale of the bottleneck accumulator
+
+// Logistic function with the hardware exponential and divide: these sit on the
+// per-step critical path (relative error ~1e-6, far inside the parity bounds).
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// tanh(x) = 2 sigmoid(2x) - 1
+__device__ __forceinline__ float tanh_fast(float x) { return fmaf(2.f, sigmoid_fast(2.f * x), -1.f); }
 
 // Consumer warps per CTA for a request group of NB: enough warps per scheduler to
 // hide FMA / shuffle / shared-memory latency, within the register file and the
 // shared memory left beside the larger groups' per-request state.
-template <int NB> struct Warps { static constexpr int NCW = NB <= 2 ? 12 : (NB == 4 ? 8 : 4); };
-constexpr int ncw_of(int NB) { return NB <= 2 ? 12 : (NB == 4 ? 8 : 4); }
+template <int NB> struct Warps { static constexpr int NCW = NB == 1 ? 12 : (NB <= 4 ? 8 : 4); };
+constexpr int ncw_of(int NB) { return NB == 1 ? 12 : (NB <= 4 ? 8 : 4); }
 
 struct Partition {
   int j0, j1;  // GRU units
@@ -247,13 +253,23 @@ __device__ void producer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     for (int c = 0; c < it.ncopy; ++c) bulk_prefetch_l2(it.src[c], it.bytes);
     ahead.next(sc, a.K);
   }
-  int n = 0, slot = 0;
+  int n = 0, n_ahead = L2_AHEAD, slot = 0;
   uint32_t phase = 0;
+  // one more L2 prefetch, at most L2_AHEAD items beyond the ring's next item
+  auto prefetch_one = [&]() {
+    if (ahead.step < a.K && n_ahead < n + L2_AHEAD) {
+      const Item& ah = table[ahead.q];
+      for (int c = 0; c < ah.ncopy; ++c) bulk_prefetch_l2(ah.src[c], ah.bytes);
+      ahead.next(sc, a.K);
+      ++n_ahead;
+    }
+  };
   for (; cur.step < a.K; ++n, cur.next(sc, a.K)) {
     if (n >= nslot) {
       const uint64_t t0 = globaltimer_ns();
       bool ok = true;
       while (!mbar_try_wait(&sh.empty[slot], phase ^ 1u)) {
+        prefetch_one();             // keep HBM busy while the consumers are held up
         if (aborted(sh)) { ok = false; break; }
         if (globaltimer_ns() - t0 > a.budget_ns) {
           raise_error(a.ctl, ERRBIT_TIMEOUT);
@@ -264,11 +280,7 @@ __device__ void producer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       }
       if (!ok) break;
     }
-    if (ahead.step < a.K) {
-      const Item& ah = table[ahead.q];
-      for (int c = 0; c < ah.ncopy; ++c) bulk_prefetch_l2(ah.src[c], ah.bytes);
-      ahead.next(sc, a.K);
-    }
+    prefetch_one();
     const Item& it = table[cur.q];
     uint8_t* dst = sh.ring + static_cast<size_t>(slot) * kLoopSlotBytes;
     mbar_arrive_expect_tx(&sh.full[slot], it.bytes * it.ncopy);
@@ -489,9 +501,9 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
           for (int g = 0; g < 3; ++g) gi[g] += sh.part_ih[(jl * sc.e3.n + s) * 32 + g * NB + b];
         for (int s = 0; s < sc.h3.n; ++s)
           for (int g = 0; g < 3; ++g) gh[g] += sh.part_hh[(jl * sc.h3.n + s) * 32 + g * NB + b];
-        const float r = 1.f / (1.f + expf(-(gi[0] + gh[0])));
-        const float z = 1.f / (1.f + expf(-(gi[1] + gh[1])));
-        const float nn = tanhf(gi[2] + r * gh[2]);
+        const float r = sigmoid_fast(gi[0] + gh[0]);
+        const float z = sigmoid_fast(gi[1] + gh[1]);
+        const float nn = tanh_fast(gi[2] + r * gh[2]);
         const float s_old = sh.S[b * a.H + j];
         const float s_new = (1.f - z) * nn + z * s_old;
         S_new[b * a.H + j] = s_new;
@@ -530,7 +542,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
         const int b = q / a.r, k = q % a.r;
         const long long fx = __ldcg(uacc_at(a, buf, b, k));
         const float pre = static_cast<float>(static_cast<double>(fx) * (1.0 / 4294967296.0));
-        sh.u[b * a.r + k] = pre / (1.f + expf(-pre));
+        sh.u[b * a.r + k] = pre * sigmoid_fast(pre);
       }
     }
     cp_async_wait_all();
@@ -613,7 +625,14 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     if (tid < nb && !aborted(sh)) {
       uint64_t k = 0;
       for (int w = 0; w < NCW; ++w) k = max(k, sh.wbest[w * NB + tid]);
-      if (k != 0ull) atomicMax(reinterpret_cast<unsigned long long*>(&a.best[i * NB + tid]), static_cast<unsigned long long>(k));
+      if (k != 0ull) {
+        atomicMax(reinterpret_cast<unsigned long long*>(&a.best[i * NB + tid]), static_cast<unsigned long long>(k));
+        // this CTA's candidate may win: bring its embedding row to L2 for the next gather
+        if (i + 1 < K && !a.forced)
+          bulk_prefetch_l2(static_cast<const uint8_t*>(a.embed) +
+                               static_cast<size_t>(argmax_key_index(k)) * a.E * a.wbytes,
+                           static_cast<uint32_t>(a.E) * a.wbytes);
+      }
     }
     grid_arrive<CONS_THREADS>(a, sh);
 

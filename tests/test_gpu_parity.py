@@ -215,6 +215,17 @@ def test_full_size_b32_gumbel_sampled():
 
 
 @cuda
+@pytest.mark.parametrize("B", [2, 8])
+def test_full_size_sweep_small_batches(B):
+    cfg = synth.sweep_config(B)
+    w, m, dw = setup(cfg)
+    hidden, anchor = synth.make_hidden(cfg), synth.make_anchor(cfg)
+    gpu = run_gpu(dw, cfg, hidden, anchor, want_logits=False)
+    assert gpu["status"] == 0
+    check_against_oracle(m, cfg, hidden, anchor, gpu, rows=[0, B - 1])
+
+
+@cuda
 def test_full_size_sweep_b256_sampled():
     cfg = synth.sweep_config(256)
     w, m, dw = setup(cfg)
