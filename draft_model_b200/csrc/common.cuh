@@ -153,6 +153,16 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Order-preserving map of a float onto uint32 (larger float -> larger integer).
+__device__ __forceinline__ uint32_t orderable_u32(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -216,9 +226,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Monotone map of an fp32 score to uint32 (larger score -> larger key), joined
 // with the inverted index so that a 64-bit max prefers the lowest index on ties.
 __device__ __forceinline__ uint64_t argmax_key(float score, uint32_t idx) {
-  const uint32_t u = __float_as_uint(score);
-  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return (static_cast<uint64_t>(k) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - idx);
+  return (static_cast<uint64_t>(orderable_u32(score)) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - idx);
 }
 __device__ __forceinline__ uint32_t argmax_key_index(uint64_t key) {
   return 0xFFFFFFFFu - static_cast<uint32_t>(key & 0xFFFFFFFFull);

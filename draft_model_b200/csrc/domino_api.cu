@@ -35,7 +35,7 @@ constexpr size_t kCtlRegion = 1024;
 static_assert(sizeof(Control) + domino::kLoopMaxGrid * 4 <= kCtlRegion, "control region");
 
 struct Layout {
-  size_t ctl, skflag, base, hp, S, u, best, skp, end;      // device workspace
+  size_t ctl, skflag, base, hp, S, u, best, skp, tc, end;  // device workspace
   size_t h_hidden, h_anchor, h_forced, h_target, h_draft, h_tau, h_end;  // host-variant staging
 };
 
@@ -70,8 +70,9 @@ Layout layout_of(const domino_weights* w, int B, int K) {
   L.hp = o; o += align_up(static_cast<size_t>(B) * K * w->rank * 4);
   L.S = o; o += align_up(2ull * 8 * w->gru_hidden * 4);
   L.u = o; o += align_up(domino::uacc_bytes(w->rank));
-  L.best = o; o += align_up(static_cast<size_t>(K) * 8 * 8);
+  L.best = o; o += align_up(static_cast<size_t>(K) * (B > 8 ? B : 8) * 8);
   L.skp = o; o += align_up(domino::lm_head_sk_bytes(B * K));
+  L.tc = o; o += align_up(domino::loop_tc_scratch_bytes(B, w->embed_dim, w->gru_hidden, w->rank));
   L.end = o;
   L.h_hidden = o; o += align_up(static_cast<size_t>(B) * K * w->d_model * wb);
   L.h_anchor = o; o += align_up(static_cast<size_t>(B) * 4);
@@ -126,6 +127,36 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
   const int sms = num_sms();
   if (sms <= 0) return DOMINO_ERR_CUDA;
   const size_t wb = w->dtype == DOMINO_BF16 ? 2 : 4;
+  if (w->dtype == DOMINO_BF16 && B >= domino::kLoopTcMinBatch &&
+      domino::loop_tc_supported(w->embed_dim, w->gru_hidden, w->d_model, w->rank, w->vocab)) {
+    // larger batches: per-step tensor-core GEMMs over the whole batch
+    domino::LoopTcArgs t;
+    std::memset(&t, 0, sizeof(t));
+    t.embed = w->embed; t.w_ih = w->w_ih; t.w_hh = w->w_hh; t.b_ih = w->b_ih; t.b_hh = w->b_hh;
+    t.w1 = w->w1; t.w2 = w->w2;
+    t.base = base;
+    t.hp = reinterpret_cast<const float*>(ws + L.hp);
+    t.anchor = anchor; t.forced = forced; t.target = target;
+    t.draft = draft; t.logits = logits; t.tau = tau;
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    const int E = w->embed_dim, H = w->gru_hidden, r = w->rank;
+    char* p = ws + L.tc;
+    t.X = reinterpret_cast<__nv_bfloat16*>(p); p += al(static_cast<size_t>(B) * E * 2);
+    t.S = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(B) * H * 4);
+    t.S2 = reinterpret_cast<__nv_bfloat16*>(p); p += al(static_cast<size_t>(B) * 2 * domino::loop_tc_padded_h(H) * 2);
+    t.gi_part = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(domino::kLoopTcMaxSplits) * B * 3 * H * 4);
+    t.gh_part = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(domino::kLoopTcMaxSplits) * B * 3 * H * 4);
+    t.u_part = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(domino::kLoopTcMaxSplits) * B * r * 4);
+    t.U2 = reinterpret_cast<__nv_bfloat16*>(p);
+    t.best = reinterpret_cast<unsigned long long*>(ws + L.best);
+    t.ctl = reinterpret_cast<Control*>(ws + L.ctl);
+    t.budget_ns = g_budget_ns.load();
+    t.seed = seed;
+    t.temperature = temperature;
+    t.mode = mode;
+    t.B = B; t.K = K; t.V = w->vocab; t.d = w->d_model; t.E = E; t.H = H; t.r = r; t.num_sms = sms;
+    return from_cuda(domino::run_loop_tc(t, st));
+  }
   const int NB = domino::loop_group_size(B);
   domino::LoopArgs a;
   std::memset(&a, 0, sizeof(a));

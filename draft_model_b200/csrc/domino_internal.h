@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace domino {
@@ -71,6 +72,44 @@ size_t loop_plan(LoopArgs& a, int NB, int grid, size_t smem_cap);
 int loop_group_size(int B);
 int loop_threads(int NB);
 cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaStream_t stream);
+
+// Stage 2 for larger batches on the tensor cores (bf16 weights), loop_tc.cu.
+constexpr int kLoopTcMinBatch = 4;     // batches from this size take the tensor-core path
+constexpr int kLoopTcMaxSplits = 8;    // split-K partial buffers of the gate and bottleneck GEMMs
+struct LoopTcArgs {
+  const void* embed; const void* w_ih; const void* w_hh; const float* b_ih; const float* b_hh;
+  const void* w1; const void* w2;
+  const float* base;       // [B, K, V]
+  const float* hp;         // [B, K, r]
+  const int32_t* anchor; const int32_t* forced; const int32_t* target;
+  int32_t* draft; float* logits; int32_t* tau;
+  // scratch
+  __nv_bfloat16* X;        // [B, E]   embeddings of the fed tokens
+  float* S;                // [B, H]   GRU state
+  __nv_bfloat16* S2;       // [B, 2*Hp] bf16 hi | lo halves of S, each padded to Hp columns
+  float* gi_part;          // [kLoopTcMaxSplits, B, 3H]
+  float* gh_part;          // [kLoopTcMaxSplits, B, 3H]
+  float* u_part;           // [kLoopTcMaxSplits, B, r]
+  __nv_bfloat16* U2;       // [2B, r]  interleaved bf16 hi / lo rows of u
+  unsigned long long* best;  // [K, B]
+  Control* ctl;
+  uint64_t budget_ns, seed;
+  float temperature;
+  int mode, B, K, V, d, E, H, r, num_sms;
+};
+cudaError_t run_loop_tc(const LoopTcArgs& args, cudaStream_t stream);
+// Shapes the tensor-core path accepts (16-byte aligned tensor-map strides, < 2^16 vocabulary tiles).
+bool loop_tc_supported(int E, int H, int d, int r, int V);
+// H rounded up to whole 64-wide k-blocks: each bf16 half of S2 has this many columns.
+inline int loop_tc_padded_h(int H) { return (H + 63) / 64 * 64; }
+// Workspace bytes of the tensor-core path's scratch for batch B.
+inline size_t loop_tc_scratch_bytes(int B, int E, int H, int r) {
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t Hp = static_cast<size_t>(loop_tc_padded_h(H));
+  return al(static_cast<size_t>(B) * E * 2) + al(static_cast<size_t>(B) * H * 4) + al(static_cast<size_t>(B) * 2 * Hp * 2) +
+         2 * al(static_cast<size_t>(kLoopTcMaxSplits) * B * 3 * H * 4) +
+         al(static_cast<size_t>(kLoopTcMaxSplits) * B * r * 4) + al(static_cast<size_t>(2) * B * r * 2);
+}
 
 // LM head (stage 1).
 // out [M, V] = hidden . W_lm^T (skipped if out is null); out2 [M, rows2] =
