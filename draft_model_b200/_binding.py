@@ -49,6 +49,7 @@ def load_library() -> ctypes.CDLL:
     sig = {
         "domino_workspace_bytes": (SZ, [W, I32, I32]),
         "domino_workspace_bytes_host": (SZ, [W, I32, I32]),
+        "domino_launches_per_block": (I32, [W, I32, I32]),
         "domino_workspace_init": (I32, [P, SZ, P]),
         "domino_draft_block": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
         "domino_draft_block_events": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P,
@@ -135,6 +136,10 @@ def domino_workspace_bytes(w: DominoWeights, B: int, K: int) -> int:
 
 def domino_workspace_bytes_host(w: DominoWeights, B: int, K: int) -> int:
     return int(load_library().domino_workspace_bytes_host(w.ref, B, K))
+
+
+def domino_launches_per_block(w: DominoWeights, B: int, K: int) -> int:
+    return int(load_library().domino_launches_per_block(w.ref, B, K))
 
 
 def domino_workspace_init(workspace: torch.Tensor, stream=None) -> None:

@@ -120,6 +120,13 @@ domino_status run_lm_head(const domino_weights* w, const void* hidden, int B, in
   return from_cuda(e);
 }
 
+// Stage 2 takes the per-step tensor-core path for bf16 batches from
+// kLoopTcMinBatch requests on shapes it supports, else the persistent loop.
+bool use_loop_tc(const domino_weights* w, int B) {
+  return w->dtype == DOMINO_BF16 && B >= domino::kLoopTcMinBatch &&
+         domino::loop_tc_supported(w->embed_dim, w->gru_hidden, w->d_model, w->rank, w->vocab);
+}
+
 domino_status run_loop(const domino_weights* w, const void* hidden, const float* base, const int32_t* anchor, int B,
                        int K, int mode, float temperature, uint64_t seed, const int32_t* forced,
                        const int32_t* target, int32_t* draft, float* logits, int32_t* tau, char* ws, const Layout& L,
@@ -127,8 +134,7 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
   const int sms = num_sms();
   if (sms <= 0) return DOMINO_ERR_CUDA;
   const size_t wb = w->dtype == DOMINO_BF16 ? 2 : 4;
-  if (w->dtype == DOMINO_BF16 && B >= domino::kLoopTcMinBatch &&
-      domino::loop_tc_supported(w->embed_dim, w->gru_hidden, w->d_model, w->rank, w->vocab)) {
+  if (use_loop_tc(w, B)) {
     // larger batches: per-step tensor-core GEMMs over the whole batch
     domino::LoopTcArgs t;
     std::memset(&t, 0, sizeof(t));
@@ -234,6 +240,16 @@ size_t domino_workspace_bytes(const domino_weights* w, int32_t B, int32_t K) {
 size_t domino_workspace_bytes_host(const domino_weights* w, int32_t B, int32_t K) {
   if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return 0;
   return layout_of(w, B, K).h_end;
+}
+
+int32_t domino_launches_per_block(const domino_weights* w, int32_t B, int32_t K) {
+  if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return -1;
+  if (use_loop_tc(w, B)) {
+    const int chunks = (B + domino::kLoopTcReqPerLaunch - 1) / domino::kLoopTcReqPerLaunch;
+    return 1 /* LM head */ + 1 /* anchor embeddings */ + K * (domino::kLoopTcLaunchesPerStep + chunks);
+  }
+  const int NB = domino::loop_group_size(B);
+  return 1 /* LM head */ + (B + NB - 1) / NB;
 }
 
 domino_status domino_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {

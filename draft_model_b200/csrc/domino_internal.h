@@ -76,6 +76,8 @@ cudaError_t launch_correct_loop(LoopArgs a, int NB, int grid, size_t smem, cudaS
 // Stage 2 for larger batches on the tensor cores (bf16 weights), loop_tc.cu.
 constexpr int kLoopTcMinBatch = 4;     // batches from this size take the tensor-core path
 constexpr int kLoopTcMaxSplits = 8;    // split-K partial buffers of the gate and bottleneck GEMMs
+constexpr int kLoopTcReqPerLaunch = 128;  // requests per W2 GEMM launch (one 256-column tile)
+constexpr int kLoopTcLaunchesPerStep = 5; // gate GEMM, GRU, bottleneck GEMM, SiLU, pick (+ W2 per chunk)
 struct LoopTcArgs {
   const void* embed; const void* w_ih; const void* w_hh; const float* b_ih; const float* b_hh;
   const void* w1; const void* w2;

@@ -32,7 +32,7 @@ namespace {
 using namespace tc;
 constexpr int EPI_WARPS = 16;                // four warps per TMEM lane quarter
 constexpr int NTH = 64 + 32 * EPI_WARPS;     // producer, MMA issuer, epilogue
-constexpr int MAXREQ_TILE = 128;             // requests per W2 tile (2 columns each)
+constexpr int MAXREQ_TILE = kLoopTcReqPerLaunch;   // requests per W2 tile (2 columns each)
 constexpr int MAX_ACC = 8;                   // TMEM accumulator buffers (as many as fit in 512 columns)
 constexpr int NSLOT = 4;                     // L_base staging ring depth (items of 8 requests)
 constexpr uint32_t SLOT_BYTES = EPI_WARPS * 8 * 32 * 4;   // 16 KB: [warp][request][lane] fp32

@@ -98,6 +98,14 @@ typedef struct {
  * the arguments are invalid. */
 DOMINO_API size_t domino_workspace_bytes(const domino_weights* w, int32_t B, int32_t K);
 
+/* Number of kernels one domino_draft_block call launches for batch B and block
+ * K (the LM head, the correction loop's kernels with verification fused into
+ * them; asynchronous memsets not counted), or -1 if the arguments are invalid.
+ * Host-only: no CUDA call.  Batches of bf16 weights from 4 requests (and
+ * 16-byte aligned E, H, d, r) take the per-step tensor-core loop; the rest take
+ * the persistent loop, one launch per group of up to 8 requests. */
+DOMINO_API int32_t domino_launches_per_block(const domino_weights* w, int32_t B, int32_t K);
+
 /* Zero the workspace control block (error word, barrier and flag counters).
  * Call once after allocating a workspace; domino_poll re-initialises it after
  * reporting a device error. */
@@ -115,7 +123,7 @@ DOMINO_API domino_status domino_workspace_init(void* workspace, size_t workspace
  *   draft_out   [B, K] int32: picked tokens t_1..t_K
  *   logits_out  [B, K, V] f32 or NULL: final logits L_i (before T and noise)
  *   tau_out     [B] int32: acceptance length; required iff target != NULL
- * Launches: LM head, correction loop (verification fused into its tail). */
+ * Launches: see domino_launches_per_block. */
 DOMINO_API domino_status domino_draft_block(const domino_weights* w, const void* hidden, const int32_t* anchor,
                                  int32_t B, int32_t K, int32_t mode, float temperature, uint64_t seed,
                                  const int32_t* forced, const int32_t* target, int32_t* draft_out,

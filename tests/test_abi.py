@@ -63,6 +63,21 @@ def test_workspace_bytes(lib):
     assert lib.domino_workspace_bytes(ctypes.byref(bad), 1, 16) == 0
 
 
+def test_launches_per_block(lib):
+    w = _cw()
+    # persistent loop: LM head + one launch per group of up to 8 requests
+    assert lib.domino_launches_per_block(ctypes.byref(w), 1, 16) == 2
+    assert lib.domino_launches_per_block(ctypes.byref(w), 2, 16) == 2
+    # tensor-core loop: LM head + anchor gather + per step 5 kernels and one W2 GEMM per 128 requests
+    assert lib.domino_launches_per_block(ctypes.byref(w), 8, 16) == 2 + 16 * 6
+    assert lib.domino_launches_per_block(ctypes.byref(w), 256, 16) == 2 + 16 * 7
+    # fp32 weights always take the persistent loop
+    wf = _cw(dtype=1)
+    assert lib.domino_launches_per_block(ctypes.byref(wf), 17, 4) == 1 + 3
+    assert lib.domino_launches_per_block(ctypes.byref(w), 0, 16) == -1
+    assert lib.domino_launches_per_block(ctypes.byref(w), 1, 33) == -1
+
+
 def _block(lib, w, *, B=1, K=16, mode=0, T=1.0, hidden=0x20000, anchor=0x30000, draft=0x40000, target=None,
            tau=None, ws=0x100000, wsn=1 << 40):
     return lib.domino_draft_block(ctypes.byref(w), hidden, anchor, B, K, mode, T, 0, None, target, draft, None, tau,
