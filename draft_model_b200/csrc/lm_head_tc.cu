@@ -94,6 +94,22 @@ __device__ __forceinline__ SegIter seg_begin(const TcArgs& a, int ntiles) {
   return it;
 }
 
+// Tile t -> (operand, vocabulary tile, position tile).  The second A operand's
+// tiles come first so they never land in the stream-K tail.  W_lm tiles run with
+// the position tile slowest: CTAs on different position tiles then stream the
+// same W_lm rows at about the same time, and the repeats are L2 hits.
+__device__ __forceinline__ void tile_decode(const TcArgs& a, int ntiles2, int t, bool& second, int& vt, int& mt) {
+  second = t < ntiles2;
+  if (second) {
+    vt = t / a.num_mt;
+    mt = t % a.num_mt;
+  } else {
+    const int tt = t - ntiles2;
+    mt = tt / a.num_vt;
+    vt = tt % a.num_vt;
+  }
+}
+
 __global__ void __launch_bounds__(NTH, 1)
     lm_head_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                       const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
@@ -140,6 +156,7 @@ __global__ void __launch_bounds__(NTH, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   auto bounded_wait = [&](uint64_t* bar, uint32_t par) -> bool {
+    if (mbar_try_wait(bar, par)) return true;   // fast path: no timer read
     if (*abort_flag) return false;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, par)) {
@@ -157,17 +174,18 @@ __global__ void __launch_bounds__(NTH, 1)
     // ---------------- TMA producer
     if (lane == 0) {
       int it = 0;  // global k-stage counter
+      int s = 0;   // ring slot of k-stage it
+      uint32_t ph = 0;  // (it / stages) & 1
       bool ok = true;
       SegIter si = seg_begin(a, ntiles);
       Seg g;
       while (ok && si.next(a, ntiles, g)) {
-        const bool second = g.t < ntiles2;
-        const int tt = second ? g.t : g.t - ntiles2;
-        const int vt = tt / a.num_mt, mt = tt % a.num_mt;
+        bool second;
+        int vt, mt;
+        tile_decode(a, ntiles2, g.t, second, vt, mt);
         const CUtensorMap* tA = second ? &tmA2 : &tmA;
         for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
-          const int s = it % a.stages;
-          if (it >= a.stages && !bounded_wait(&empty[s], ((it / a.stages) - 1) & 1)) { ok = false; break; }
+          if (it >= a.stages && !bounded_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
           uint8_t* sa = smem + static_cast<size_t>(s) * stage_bytes;
           uint8_t* sb = sa + a_bytes;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
@@ -176,6 +194,7 @@ __global__ void __launch_bounds__(NTH, 1)
             tma_load_2d(sa + j * A_STAGE_BYTES, tA, kc, vt * BM, &full[s]);
             tma_load_2d(sb + j * b_sub_bytes, &tmB, kc, mt * a.BN, &full[s]);
           }
+          if (++s == a.stages) { s = 0; ph ^= 1u; }
         }
       }
       // drain copies that were issued but may still be in flight
@@ -190,7 +209,8 @@ __global__ void __launch_bounds__(NTH, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(a.BN);
-      int it = 0, local = 0;
+      int it = 0, local = 0, s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       SegIter si = seg_begin(a, ntiles);
       Seg g;
@@ -200,20 +220,20 @@ __global__ void __launch_bounds__(NTH, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
         for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
-          const int s = it % a.stages;
-          if (!bounded_wait(&full[s], (it / a.stages) & 1)) { ok = false; break; }
+          if (!bounded_wait(&full[s], ph)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-          const uint32_t sb = sa + a_bytes;
+          // descriptors advance by (bytes >> 4) in their start-address field
+          const uint64_t da = smem_desc_sw128(smem_u32(smem + static_cast<size_t>(s) * stage_bytes));
+          const uint64_t db = da + (a_bytes >> 4);
           for (int j = 0; j < a.nk; ++j) {
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              tc_mma_bf16(d_tmem, smem_desc_sw128(sa + j * A_STAGE_BYTES + kk * 32),
-                          smem_desc_sw128(sb + j * b_sub_bytes + kk * 32), idesc,
-                          (kb > g.kb0 || j > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_bf16(d_tmem, da + ((j * A_STAGE_BYTES + kk * 32) >> 4), db + ((j * b_sub_bytes + kk * 32) >> 4),
+                          idesc, (kb > g.kb0 || j > 0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit(&empty[s]);   // frees the stage once these MMAs have read it
+          if (++s == a.stages) { s = 0; ph ^= 1u; }
         }
         if (ok) tc_commit(&tfull[acc]);
         ++local;
@@ -237,9 +257,9 @@ __global__ void __launch_bounds__(NTH, 1)
       named_barrier(2, 128);          // the four epilogue warps take the same decision
       if (*abort_flag) break;
       tc_fence_after();
-      const bool second = g.t < ntiles2;
-      const int tt = second ? g.t : g.t - ntiles2;
-      const int vt = tt / a.num_mt, mt = tt % a.num_mt;
+      bool second;
+      int vt, mt;
+      tile_decode(a, ntiles2, g.t, second, vt, mt);
       const int row = q * 32 + lane;                 // row of the 128-row tile
       const int v = vt * BM + row;
       const int nrows = second ? a.rows2 : a.V;

@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(NTH, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   auto bounded_wait = [&](uint64_t* bar, uint32_t par) -> bool {
+    if (mbar_try_wait(bar, par)) return true;   // fast path: no timer read
     if (*abort_flag) return false;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, par)) {
@@ -167,7 +168,8 @@ __global__ void __launch_bounds__(NTH, 1)
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
-      int it = 0;
+      int it = 0, s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
         int pi, vt, mt, kb0, kb1, split;
@@ -176,13 +178,13 @@ __global__ void __launch_bounds__(NTH, 1)
         const CUtensorMap* tB = pi == 0 ? &tmB0 : &tmB1;
         const int wrap = a.p[pi].a_kwrap;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % a.stages;
-          if (it >= a.stages && !bounded_wait(&empty[s], ((it / a.stages) - 1) & 1)) { ok = false; break; }
+          if (it >= a.stages && !bounded_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
           uint8_t* sa = smem + static_cast<size_t>(s) * stage_bytes;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
           const int kc = kb * BK;
           tma_load_2d(sa, tA, wrap ? kc % wrap : kc, vt * BM, &full[s]);
           tma_load_2d(sa + A_STAGE_BYTES, tB, kc, mt * a.BN, &full[s]);
+          if (++s == a.stages) { s = 0; ph ^= 1u; }
         }
       }
       for (int j = max(0, it - a.stages); j < it; ++j) {
@@ -196,7 +198,8 @@ __global__ void __launch_bounds__(NTH, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(a.BN);
-      int it = 0, local = 0;
+      int it = 0, local = 0, s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x, ++local) {
         int pi, vt, mt, kb0, kb1, split;
@@ -206,15 +209,16 @@ __global__ void __launch_bounds__(NTH, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % a.stages;
-          if (!bounded_wait(&full[s], (it / a.stages) & 1)) { ok = false; break; }
+          if (!bounded_wait(&full[s], ph)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+          // descriptors advance by (bytes >> 4) in their start-address field
+          const uint64_t da = smem_desc_sw128(smem_u32(smem + static_cast<size_t>(s) * stage_bytes));
+          const uint64_t db = da + (A_STAGE_BYTES >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_bf16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sa + A_STAGE_BYTES + kk * 32), idesc,
-                        (kb > kb0 || kk > 0) ? 1u : 0u);
+            tc_mma_bf16(d_tmem, da + ((kk * 32) >> 4), db + ((kk * 32) >> 4), idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
+          if (++s == a.stages) { s = 0; ph ^= 1u; }
         }
         if (ok) tc_commit(&tfull[acc]);
       }

@@ -44,7 +44,10 @@ def setup(cfg):
 @pytest.mark.parametrize("B,K,d,V", [(1, 16, 256, 1000), (3, 5, 200, 5000), (20, 16, 136, 777), (1, 4, 64, 128),
                                      (2, 16, 4096, 3000),
                                      # more 128-row tiles than SMs, ragged: stream-K splits tiles across CTAs
-                                     (1, 16, 512, 30000), (1, 16, 1032, 20011), (3, 16, 256, 40000)])
+                                     (1, 16, 512, 30000), (1, 16, 1032, 20011), (3, 16, 256, 40000),
+                                     # 256 block positions per tile: vocabulary tiles run in pairs
+                                     # (odd tile count -> a half-empty last pair), with stream-K
+                                     (16, 16, 512, 40000), (20, 16, 264, 20011)])
 def test_lm_head_bf16_tcgen05(B, K, d, V):
     cfg = small(B=B, K=K, d=d, V=V)
     w, m, dw = setup(cfg)
