@@ -285,19 +285,32 @@ __global__ void __launch_bounds__(NTH, 1)
       }
       const float* park_in = a.sk_part + static_cast<size_t>(blockIdx.x + 1) * a.BN * BM;
       float* park_out = a.sk_part + static_cast<size_t>(blockIdx.x) * a.BN * BM;
-      for (int c0 = 0; c0 < a.BN; c0 += 16) {
-        float vals[16];
-        tmem_ld16(trow + c0, vals);
+      for (int cb = 0; cb < a.BN; cb += 64) {
+        // a HEAD adds the parked tail: its 64 columns are loaded together, before
+        // any store of this batch (the stores could alias them for the compiler,
+        // which would otherwise serialise one load latency per column)
+        float part[64];
+        if (g.kind == SEG_HEAD) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int col = c0 + c;
-          if (g.kind == SEG_TAIL) {
-            park_out[static_cast<size_t>(col) * BM + row] = vals[c];
-          } else {
-            float x = vals[c];
-            if (g.kind == SEG_HEAD) x += __ldcg(park_in + static_cast<size_t>(col) * BM + row);
-            const int m = mt * a.BN + col;
-            if (v < nrows && m < a.M) dst[static_cast<size_t>(m) * nrows + v] = x;
+          for (int c = 0; c < 64; ++c)
+            part[c] = cb + c < a.BN ? __ldcg(park_in + static_cast<size_t>(cb + c) * BM + row) : 0.f;
+        }
+#pragma unroll
+        for (int c1 = 0; c1 < 64; c1 += 16) {
+          const int c0 = cb + c1;
+          if (c0 >= a.BN) break;
+          float vals[16];
+          tmem_ld16(trow + c0, vals);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int col = c0 + c;
+            if (g.kind == SEG_TAIL) {
+              park_out[static_cast<size_t>(col) * BM + row] = vals[c];
+            } else {
+              const float x = g.kind == SEG_HEAD ? vals[c] + part[c1 + c] : vals[c];
+              const int m = mt * a.BN + col;
+              if (v < nrows && m < a.M) dst[static_cast<size_t>(m) * nrows + v] = x;
+            }
           }
         }
       }
