@@ -158,6 +158,14 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Programmatic dependent launch (kernels launched with programmatic stream
+// serialization): let the next kernel in the stream start its prologue now, and
+// wait until the kernel this one depends on has completed and its writes are
+// visible.  Both are no-ops for a normally launched kernel.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Order-preserving map of a float onto uint32 (larger float -> larger integer).
 __device__ __forceinline__ uint32_t orderable_u32(float x) {
   const uint32_t u = __float_as_uint(x);

@@ -21,6 +21,7 @@
 // summed in a fixed order; the argmax merge is order-free).
 #include <cstdint>
 #include <cstring>
+#include <utility>
 
 #include "common.cuh"
 #include "domino_internal.h"
@@ -149,6 +150,10 @@ __global__ void __launch_bounds__(NTH, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the setup above overlaps the previous kernel of the step chain; every global
+  // access below comes after it has completed
+  griddep_launch_dependents();
+  griddep_wait();
 
   auto bounded_wait = [&](uint64_t* bar, uint32_t par) -> bool {
     if (mbar_try_wait(bar, par)) return true;   // fast path: no timer read
@@ -390,6 +395,8 @@ __global__ void __launch_bounds__(256) gru_step_kernel(const float* __restrict__
                                                        const float* __restrict__ b_ih, const float* __restrict__ b_hh,
                                                        float* __restrict__ S, __nv_bfloat16* __restrict__ S2, int B,
                                                        int H, int Hp) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * H) return;
   const int b = idx / H, j = idx % H;
@@ -424,6 +431,8 @@ __global__ void __launch_bounds__(256) gru_step_kernel(const float* __restrict__
 __global__ void __launch_bounds__(256) silu_split_kernel(const float* __restrict__ upart, int splits,
                                                          const float* __restrict__ hp, int K, int step, int B, int r,
                                                          __nv_bfloat16* __restrict__ U2) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * r) return;
   const int b = idx / r, k = idx % r;
@@ -446,6 +455,8 @@ __global__ void __launch_bounds__(256) pick_step_kernel(unsigned long long* best
                                                         int32_t* tau, const __nv_bfloat16* __restrict__ embed,
                                                         __nv_bfloat16* X, Control* ctl) {
   // one block per request: thread 0 decides the token, all threads copy the row
+  griddep_launch_dependents();
+  griddep_wait();
   const int b = blockIdx.x;
   __shared__ int fed;
   if (threadIdx.x == 0) {
@@ -499,6 +510,24 @@ GemmKernel gemm_kernel(int epi) {
     case EPI_GUMBEL_LOGITS: return gemm_tc_kernel<EPI_GUMBEL_LOGITS>;
     default: return gemm_tc_kernel<EPI_PARTIAL>;
   }
+}
+
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous one finishes; it calls griddep_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
@@ -572,9 +601,9 @@ cudaError_t run_loop_tc(const LoopTcArgs& L, cudaStream_t st) {
   if ((e = cudaMemsetAsync(L.S, 0, static_cast<size_t>(B) * H * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(L.S2, 0, static_cast<size_t>(B) * 2 * Hp * 2, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(L.best, 0, static_cast<size_t>(K) * B * 8, st)) != cudaSuccess) return e;
-  pick_step_kernel<<<B, 256, 0, st>>>(L.best, -1, K, B, V, E, L.anchor, L.forced, L.target, L.draft, L.tau,
-                                      static_cast<const __nv_bfloat16*>(L.embed), L.X, L.ctl);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_pdl(pick_step_kernel, dim3(B), dim3(256), 0, st, L.best, -1, K, B, V, E, L.anchor, L.forced, L.target,
+                 L.draft, L.tau, static_cast<const __nv_bfloat16*>(L.embed), L.X, L.ctl);
+  if (e != cudaSuccess) return e;
 
   for (int i = 0; i < K; ++i) {
     // 1. gate GEMMs (W_hh S is zero at the first position: S = 0)
@@ -582,17 +611,18 @@ cudaError_t run_loop_tc(const LoopTcArgs& L, cudaStream_t st) {
     g.units0 = vt * num_mt * s0;
     g.units = g.units0 + (i == 0 ? 0 : vt * num_mt * s1);
     const int grid0 = g.units < L.num_sms ? g.units : L.num_sms;
-    gemm_tc_kernel<EPI_PARTIAL><<<grid0, NTH, gsm, st>>>(tWih, tX, tWhh, tS2, g);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(gemm_tc_kernel<EPI_PARTIAL>, dim3(grid0), dim3(NTH), gsm, st, tWih, tX, tWhh, tS2, g);
+    if (e != cudaSuccess) return e;
     // 2. GRU
-    gru_step_kernel<<<(B * H + 255) / 256, 256, 0, st>>>(L.gi_part, s0, L.gh_part, i == 0 ? 0 : s1, L.b_ih, L.b_hh,
-                                                        L.S, L.S2, B, H, Hp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(gru_step_kernel, dim3((B * H + 255) / 256), dim3(256), 0, st, L.gi_part, s0, L.gh_part,
+                   i == 0 ? 0 : s1, L.b_ih, L.b_hh, L.S, L.S2, B, H, Hp);
+    if (e != cudaSuccess) return e;
     // 3. bottleneck product, 4. SiLU and the hi / lo split of u
-    gemm_tc_kernel<EPI_PARTIAL><<<gridb, NTH, gsm, st>>>(tW1s, tS2, tW1s, tS2, bk);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    silu_split_kernel<<<(B * r + 255) / 256, 256, 0, st>>>(L.u_part, pb.splits, L.hp, K, i, B, r, L.U2);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(gemm_tc_kernel<EPI_PARTIAL>, dim3(gridb), dim3(NTH), gsm, st, tW1s, tS2, tW1s, tS2, bk);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(silu_split_kernel, dim3((B * r + 255) / 256), dim3(256), 0, st, L.u_part, pb.splits, L.hp, K, i, B,
+                   r, L.U2);
+    if (e != cudaSuccess) return e;
     // 5. W2 GEMM + residual + pick, per chunk of requests
     for (int c0 = 0; c0 < B; c0 += MAXREQ_TILE) {
       const int nreq = B - c0 < MAXREQ_TILE ? B - c0 : MAXREQ_TILE;
@@ -617,13 +647,13 @@ cudaError_t run_loop_tc(const LoopTcArgs& L, cudaStream_t st) {
       w.temperature = L.temperature;
       w.seed = L.seed;
       const int gridw = w.units < L.num_sms ? w.units : L.num_sms;
-      gemm_kernel(epi_w2)<<<gridw, NTH, wsm, st>>>(tW2, tU, tW2, tU, w);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      e = launch_pdl(gemm_kernel(epi_w2), dim3(gridw), dim3(NTH), wsm, st, tW2, tU, tW2, tU, w);
+      if (e != cudaSuccess) return e;
     }
     // 6. picks, next fed tokens and embeddings (verification after the last position)
-    pick_step_kernel<<<B, 256, 0, st>>>(L.best, i, K, B, V, E, L.anchor, L.forced, L.target, L.draft, L.tau,
-                                        static_cast<const __nv_bfloat16*>(L.embed), L.X, L.ctl);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(pick_step_kernel, dim3(B), dim3(256), 0, st, L.best, i, K, B, V, E, L.anchor, L.forced, L.target,
+                   L.draft, L.tau, static_cast<const __nv_bfloat16*>(L.embed), L.X, L.ctl);
+    if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
