@@ -382,7 +382,11 @@ def run_ours(args):
     achieved = lbytes / loop_avg / 1e9
     traffic = recorded_traffic("correct_loop_kernel") if B == 1 else None
     lm_frac_hbm = lm_head_bytes(cfg, B) / lm_avg / 1e9 / peaks["hbm_gbs"]
-    lm_frac_tc = lm_head_flops(cfg, B) / lm_avg / 1e12 / peaks["bf16_tflops"]
+    lm_tflops = lm_head_flops(cfg, B) / lm_avg / 1e12
+    # the LM head runs inside a long back-to-back step: the sustained (power-capped)
+    # GEMM peak is its denominator; the burst figure is reported beside it
+    lm_frac_tc = lm_tflops / peaks["bf16_tflops_sustained"]
+    lm_frac_tc_burst = lm_tflops / peaks["bf16_tflops"]
     launches = dm.domino_launches_per_block(dw, B, cfg.K)
     persistent = launches == 1 + -(-B // min(8, 1 << (B.bit_length() - 1)))
 
@@ -410,7 +414,9 @@ def run_ours(args):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "algorithmic_bytes": lbytes, "peak_source": peak_kind},
         "lm_head_roofline": {"bound": "hbm" if B < 32 else "tensor", "frac_of_hbm": lm_frac_hbm,
-                             "frac_of_bf16_tensor": lm_frac_tc, "peak_source": peak_kind},
+                             "achieved_tflops": lm_tflops,
+                             "frac_of_bf16_tensor": lm_frac_tc, "tensor_peak": "bf16_tflops_sustained",
+                             "frac_of_bf16_tensor_burst": lm_frac_tc_burst, "peak_source": peak_kind},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * launches,
