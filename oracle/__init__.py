@@ -10,10 +10,14 @@ vectors; the GRU step against torch.nn.GRUCell and a hand-computed closed form;
 SiLU against its closed form; the LM head against a brute-force triple loop;
 zero-correction invariants; teacher-forcing and causality invariants; a
 brute-force greedy fixed point; the exact Gumbel-max law; tau by brute force;
-the head's parameter count against the pages' "56M".
+the head's parameter count against the pages' "56M"; the training loss's
+cross-entropy against torch's and closed forms (uniform rows, two-way rows),
+its curriculum mix and position weights against their limits.
 """
 from .domino_ref import Model, Result, draft_block, gru_cell, lm_head, positions, sigmoid, silu, verify, widen_f64
 from .philox import gumbel_noise, philox4x32_10, philox4x32_10_np, uniform_from_word
+from .training import cross_entropy_rows, curriculum_loss, position_weights, train_forward
 
 __all__ = ["Model", "Result", "draft_block", "gru_cell", "lm_head", "positions", "sigmoid", "silu", "verify",
-           "widen_f64", "gumbel_noise", "philox4x32_10", "philox4x32_10_np", "uniform_from_word"]
+           "widen_f64", "gumbel_noise", "philox4x32_10", "philox4x32_10_np", "uniform_from_word",
+           "cross_entropy_rows", "curriculum_loss", "position_weights", "train_forward"]
