@@ -426,6 +426,81 @@ def run_ours(args):
     barrier(world)
 
 
+def run_loss(args):
+    """Training forward (teacher-forced block + base-anchored curriculum loss) on one GPU.
+
+    Times domino_draft_loss per step (L2 flushed between steps) and, on its own,
+    the curriculum-loss kernels over [B, K, V] final and base logits against the
+    HBM roofline (both tensors read once).
+    """
+    import numpy as np
+    import torch
+
+    import draft_model_b200 as dm
+    import synth
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from _harness import aligned_workspace, device_weights, to_dev
+
+    dm.load_library()
+    B = args.batch
+    cfg = workload_config(B)
+    dw = device_weights(synth.make_weights(cfg))
+    hidden = to_dev(synth.make_hidden(cfg, B), cfg.dtype)
+    anchor = torch.from_numpy(synth.make_anchor(cfg, B)).cuda()
+    labels = torch.from_numpy(np.random.default_rng([7, B]).integers(0, cfg.V, size=(B, cfg.K)).astype(np.int32)).cuda()
+    ws = aligned_workspace(dm.domino_draft_loss_workspace_bytes(dw, B, cfg.K))
+    loss = torch.zeros(4, dtype=torch.float32, device="cuda")
+    scrub = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+    def step(k):
+        scrub.fill_(float(k))
+        e = ev[min(k, args.steps - 1)]
+        e[0].record()
+        dm.domino_draft_loss(dw, hidden, anchor, labels, lam=0.5, gamma=0.9, loss_out=loss, workspace=ws)
+        e[1].record()
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        step(k)
+    torch.cuda.synchronize()
+    if dm.domino_poll(ws) != 0:
+        raise RuntimeError("device error in the training forward")
+    t = statistics.mean(e[0].elapsed_time(e[1]) * 1e-3 for e in ev)
+
+    # the loss kernels alone on resident logits
+    fin = torch.randn((B, cfg.K, cfg.V), device="cuda") * 4
+    bas = torch.randn((B, cfg.K, cfg.V), device="cuda") * 4
+    lws = aligned_workspace(dm.domino_curriculum_loss_workspace_bytes(B, cfg.K, cfg.V))
+    lt = []
+    for k in range(args.warmup + 20):
+        scrub.fill_(float(k))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dm.domino_curriculum_loss(fin, bas, labels, lam=0.5, gamma=0.9, loss_out=loss, workspace=lws)
+        e1.record()
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            lt.append(e0.elapsed_time(e1) * 1e-3)
+    lt_avg = statistics.mean(lt)
+    peaks, peak_kind = measured_peaks()
+    ce_bytes = 2 * B * cfg.K * cfg.V * 4
+    achieved = ce_bytes / lt_avg / 1e9
+    print(json.dumps({
+        "metric": "training_forward_blocks_per_s", "value": B / t, "unit": "blocks/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD.format(B=B) + ", teacher-forced, curriculum loss lambda 0.5 gamma 0.9",
+                   "l2": "flushed before every step"},
+        "curriculum_loss_kernels": {"us": lt_avg * 1e6, "bound": "hbm", "achieved": achieved,
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                                    "algorithmic_bytes": ce_bytes, "peak_source": peak_kind},
+        "loss": float(loss[0].item()),
+    }), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -434,11 +509,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--batch", type=int, default=1, help="requests per GPU per draft block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["draft", "loss"], default="draft",
+                    help="draft: the draft block (default); loss: the teacher-forced training forward")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "loss":
+        run_loss(args)
     else:
         run_ours(args)
     _, _, world = dist_env()

@@ -50,6 +50,10 @@ def load_library() -> ctypes.CDLL:
         "domino_workspace_bytes": (SZ, [W, I32, I32]),
         "domino_workspace_bytes_host": (SZ, [W, I32, I32]),
         "domino_launches_per_block": (I32, [W, I32, I32]),
+        "domino_curriculum_loss_workspace_bytes": (SZ, [I32, I32, I32]),
+        "domino_curriculum_loss": (I32, [P, P, P, I32, I32, I32, F, F, P, P, P, SZ, P]),
+        "domino_draft_loss_workspace_bytes": (SZ, [W, I32, I32]),
+        "domino_draft_loss": (I32, [W, P, P, P, I32, I32, F, F, P, P, P, SZ, P]),
         "domino_workspace_init": (I32, [P, SZ, P]),
         "domino_draft_block": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
         "domino_draft_block_events": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P,
@@ -199,6 +203,34 @@ def domino_correct_loop_noalloc(w: DominoWeights, hidden, base, anchor, *, mode=
                                                       temperature, seed, _ptr(forced), _ptr(target),
                                                       _ptr(draft_out), _ptr(logits_out), _ptr(tau_out),
                                                       _stream(stream)), "domino_correct_loop_noalloc")
+
+
+def domino_curriculum_loss_workspace_bytes(B: int, K: int, V: int) -> int:
+    return int(load_library().domino_curriculum_loss_workspace_bytes(B, K, V))
+
+
+def domino_curriculum_loss(final_logits, base_logits, labels, *, lam: float, gamma: float, loss_out, ce_out=None,
+                           workspace, stream=None) -> None:
+    """Base-anchored curriculum loss of [B, K, V] fp32 logits against [B, K] labels."""
+    B, K, V = final_logits.shape
+    wp, wn = _ws(workspace)
+    _check(load_library().domino_curriculum_loss(_ptr(final_logits), _ptr(base_logits), _ptr(labels), B, K, V, lam,
+                                                 gamma, _ptr(ce_out), _ptr(loss_out), wp, wn, _stream(stream)),
+           "domino_curriculum_loss")
+
+
+def domino_draft_loss_workspace_bytes(w: DominoWeights, B: int, K: int) -> int:
+    return int(load_library().domino_draft_loss_workspace_bytes(w.ref, B, K))
+
+
+def domino_draft_loss(w: DominoWeights, hidden, anchor, labels, *, lam: float, gamma: float, loss_out, ce_out=None,
+                      workspace, stream=None) -> None:
+    """Teacher-forced training forward (GRU fed the labels) and its curriculum loss."""
+    B, K = labels.shape
+    wp, wn = _ws(workspace)
+    _check(load_library().domino_draft_loss(w.ref, _ptr(hidden), _ptr(anchor), _ptr(labels), B, K, lam, gamma,
+                                            _ptr(ce_out), _ptr(loss_out), wp, wn, _stream(stream)),
+           "domino_draft_loss")
 
 
 def domino_verify(draft, target, tau_out, stream=None) -> None:

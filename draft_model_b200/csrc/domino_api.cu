@@ -327,6 +327,67 @@ domino_status domino_draft_block(const domino_weights* w, const void* hidden, co
                                    logits_out, tau_out, workspace, workspace_bytes, stream, nullptr);
 }
 
+// ---------------------------------------------------------------- training forward
+
+size_t domino_curriculum_loss_workspace_bytes(int32_t B, int32_t K, int32_t V) {
+  if (B < 1 || K < 1 || K > 32 || V < 1) return 0;
+  return kCtlRegion + align_up(domino::loss_scratch_bytes(B, K, V));
+}
+
+domino_status domino_curriculum_loss(const float* final_logits, const float* base_logits, const int32_t* labels,
+                                     int32_t B, int32_t K, int32_t V, float lambda, float gamma, float* ce_out,
+                                     float* loss_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 1 || K < 1 || K > 32 || V < 1 || static_cast<long long>(B) * K > 65535 / 2) return DOMINO_ERR_INVALID_ARG;
+  if (!final_logits || !base_logits || !labels || !loss_out) return DOMINO_ERR_INVALID_ARG;
+  if (!aligned16(final_logits) || !aligned16(base_logits) || !aligned16(labels) || !aligned16(loss_out) ||
+      (ce_out && !aligned16(ce_out)))
+    return DOMINO_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f && lambda <= 1.f) || !(gamma > 0.f && std::isfinite(gamma))) return DOMINO_ERR_INVALID_ARG;
+  domino_status s = check_workspace(workspace, workspace_bytes, domino_curriculum_loss_workspace_bytes(B, K, V));
+  if (s != DOMINO_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  return from_cuda(domino::launch_curriculum_loss(final_logits, base_logits, labels, B, K, V, lambda, gamma,
+                                                  ws + kCtlRegion, ce_out, loss_out, reinterpret_cast<Control*>(ws),
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+size_t domino_draft_loss_workspace_bytes(const domino_weights* w, int32_t B, int32_t K) {
+  if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return 0;
+  const size_t rows = static_cast<size_t>(B) * K;
+  return layout_of(w, B, K).end + align_up(rows * w->vocab * 4) + align_up(rows * 4) +
+         align_up(domino::loss_scratch_bytes(B, K, w->vocab));
+}
+
+domino_status domino_draft_loss(const domino_weights* w, const void* hidden, const int32_t* anchor,
+                                const int32_t* labels, int32_t B, int32_t K, float lambda, float gamma,
+                                float* ce_out, float* loss_out, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (!labels || !loss_out || !aligned16(loss_out) || (ce_out && !aligned16(ce_out))) return DOMINO_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * K > 65535 / 2) return DOMINO_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f && lambda <= 1.f) || !(gamma > 0.f && std::isfinite(gamma))) return DOMINO_ERR_INVALID_ARG;
+  const Layout L = layout_of(w, B, K);
+  const size_t rows = static_cast<size_t>(B) * K;
+  domino_status s = check_workspace(workspace, workspace_bytes, domino_draft_loss_workspace_bytes(w, B, K));
+  if (s != DOMINO_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  float* final_logits = reinterpret_cast<float*>(ws + L.end);
+  int32_t* picks = reinterpret_cast<int32_t*>(ws + L.end + align_up(rows * w->vocab * 4));
+  void* scratch = ws + L.end + align_up(rows * w->vocab * 4) + align_up(rows * 4);
+  s = validate_block(w, hidden, anchor, B, K, DOMINO_GREEDY, 1.f, labels, nullptr, picks, final_logits, nullptr);
+  if (s != DOMINO_OK) return s;
+  if (!weight_ptrs_ok(w, true, true)) return DOMINO_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* base = reinterpret_cast<float*>(ws + L.base);
+  // teacher forcing: the labels are the GRU's inputs after each position
+  s = run_lm_head(w, hidden, B, K, base, reinterpret_cast<float*>(ws + L.hp), ws, L, st);
+  if (s != DOMINO_OK) return s;
+  s = run_loop(w, hidden, base, anchor, B, K, DOMINO_GREEDY, 1.f, 0, labels, nullptr, picks, final_logits, nullptr,
+               ws, L, st);
+  if (s != DOMINO_OK) return s;
+  return from_cuda(domino::launch_curriculum_loss(final_logits, base, labels, B, K, w->vocab, lambda, gamma, scratch,
+                                                  ce_out, loss_out, reinterpret_cast<Control*>(ws + L.ctl), st));
+}
+
 domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K, int32_t* tau_out,
                             void* stream) {
   if (!draft || !target || !tau_out || B < 1 || K < 1 || K > 32) return DOMINO_ERR_INVALID_ARG;

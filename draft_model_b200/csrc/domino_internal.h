@@ -131,6 +131,13 @@ cudaError_t launch_lm_head_f32(const float* w, const float* hidden, float* out, 
                                cudaStream_t stream);
 
 // Verification (stage 3).
+// Base-anchored curriculum loss over fp32 logit rows (loss.cu).
+int loss_chunks(int B, int K, int V);
+size_t loss_scratch_bytes(int B, int K, int V);
+cudaError_t launch_curriculum_loss(const float* final_logits, const float* base_logits, const int32_t* labels, int B,
+                                   int K, int V, float lambda, float gamma, void* scratch, float* ce_out,
+                                   float* loss_out, Control* ctl, cudaStream_t stream);
+
 cudaError_t launch_verify(const int32_t* draft, const int32_t* target, int B, int K, int32_t* tau,
                           cudaStream_t stream);
 

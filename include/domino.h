@@ -178,6 +178,45 @@ DOMINO_API domino_status domino_correct_loop_noalloc(const domino_weights* w, co
                                           int32_t* tau_out, void* stream);
 
 /* Stage 3 only: tau_out[b] = number of leading i with draft[b, i] == target[b, i]. */
+/* ---- Training forward (Domino study notes, gsyq.cn, §二.2 配套专属训练方案) ----
+ *
+ * Base-anchored curriculum loss (§二.2(2)) on given logits:
+ *   loss = (1 - lambda) L_final + lambda L_base,
+ *   L_x  = sum_{b,i} gamma^i CE(x[b,i,:], labels[b,i]) / (B sum_i gamma^i),
+ *   CE(l, y) = logsumexp(l) - l[y]   (no temperature),
+ * i = 0..K-1 the block position minus one (exponentially decaying position
+ * weights; the notes give no decay constant, gamma is the caller's).
+ *   final_logits, base_logits [B, K, V] fp32 device, 16-byte aligned
+ *   labels      [B, K] int32 ground-truth tokens; out-of-range values are
+ *               clamped and flagged (DOMINO_ERR_BAD_TOKEN via domino_poll)
+ *   lambda      in [0, 1] (the notes anneal it linearly from 1 to 0 over training)
+ *   gamma       > 0 (1 = uniform weights)
+ *   ce_out      [B, K, 2] fp32 or NULL: per-position (final, base) cross-entropy
+ *   loss_out    [1] fp32 device
+ *   workspace   domino_curriculum_loss_workspace_bytes(B, K, V) bytes, 256-byte
+ *               aligned, zeroed once with domino_workspace_init.
+ * Two launches (one CTA per row chunk, then one combining CTA); deterministic.
+ * Argument errors (NULL, misaligned, lambda or gamma out of range, B K > 32767)
+ * return synchronously. */
+DOMINO_API size_t domino_curriculum_loss_workspace_bytes(int32_t B, int32_t K, int32_t V);
+DOMINO_API domino_status domino_curriculum_loss(const float* final_logits, const float* base_logits,
+                                                const int32_t* labels, int32_t B, int32_t K, int32_t V, float lambda,
+                                                float gamma, float* ce_out, float* loss_out, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
+/* Teacher-forced training forward (§二.2(1) Teacher-Forced, §二.2(2)): one draft
+ * block per request whose GRU reads the ground truth (labels[b, i] is the
+ * target of position i+1 and the GRU input after it, i.e. domino_draft_block
+ * with forced = labels), then the curriculum loss of its final and base logits
+ * against the labels.  Arguments as for domino_draft_block and
+ * domino_curriculum_loss; the final logits are written to the workspace, whose
+ * size is domino_draft_loss_workspace_bytes(w, B, K). */
+DOMINO_API size_t domino_draft_loss_workspace_bytes(const domino_weights* w, int32_t B, int32_t K);
+DOMINO_API domino_status domino_draft_loss(const domino_weights* w, const void* hidden, const int32_t* anchor,
+                                           const int32_t* labels, int32_t B, int32_t K, float lambda, float gamma,
+                                           float* ce_out, float* loss_out, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
 DOMINO_API domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K,
                             int32_t* tau_out, void* stream);
 

@@ -45,6 +45,15 @@ def device_weights(w: synth.Weights, device="cuda") -> dm.DominoWeights:
                             to_dev(w.w1, dt, device), to_dev(w.w2, dt, device))
 
 
+def aligned_workspace(n: int) -> torch.Tensor:
+    """n bytes of 256-byte aligned device memory with a zeroed control block."""
+    ws = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + n]
+    dm.domino_workspace_init(ws)
+    return ws
+
+
 def workspace_for(dw: dm.DominoWeights, B: int, K: int, host: bool = False) -> torch.Tensor:
     n = dm.domino_workspace_bytes_host(dw, B, K) if host else dm.domino_workspace_bytes(dw, B, K)
     ws = torch.empty(n + 256, dtype=torch.uint8, device="cuda")

@@ -121,3 +121,20 @@ def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_binding, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _binding.load_library()
+
+
+def test_loss_validation_is_host_side(lib):
+    INVALID = 1
+    p = 0x100000
+    n = lib.domino_curriculum_loss_workspace_bytes(2, 4, 1000)
+    assert n > 0 and lib.domino_curriculum_loss_workspace_bytes(0, 4, 1000) == 0
+    call = lambda lam, gamma, B=2, K=4: lib.domino_curriculum_loss(p, p, p, B, K, 1000, lam, gamma, None, p, p, n, None)
+    assert call(-0.1, 1.0) == INVALID
+    assert call(1.5, 1.0) == INVALID
+    assert call(0.5, 0.0) == INVALID
+    assert call(0.5, float("inf")) == INVALID
+    assert call(0.5, 1.0, K=33) == INVALID
+    assert lib.domino_curriculum_loss(p, p, None, 2, 4, 1000, 0.5, 1.0, None, p, p, n, None) == INVALID
+    w = _cw()
+    assert lib.domino_draft_loss_workspace_bytes(ctypes.byref(w), 1, 16) > lib.domino_workspace_bytes(ctypes.byref(w), 1, 16)
+    assert lib.domino_draft_loss(ctypes.byref(w), p, p, None, 1, 16, 0.5, 1.0, None, p, p, 1 << 40, None) == INVALID
