@@ -501,6 +501,62 @@ def run_loss(args):
     }), flush=True)
 
 
+def run_verify(args):
+    """Stochastic verification (speculative sampling) of a block of the workload's shape.
+
+    Times domino_verify_sample on resident synthetic draft logits [B, K, V] and
+    target logits [B, K+1, V] (L2 flushed between launches) against the HBM
+    roofline: every row read once plus the resampled row pair read again.
+    """
+    import numpy as np
+    import torch
+
+    import draft_model_b200 as dm
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from _harness import aligned_workspace
+
+    dm.load_library()
+    B = args.batch
+    cfg = workload_config(B)
+    K, V = cfg.K, cfg.V
+    g = torch.Generator(device="cuda").manual_seed(5)
+    dl = torch.randn((B, K, V), device="cuda", generator=g) * 2
+    tl = torch.cat([dl + 0.5 * torch.randn((B, K, V), device="cuda", generator=g),
+                    2 * torch.randn((B, 1, V), device="cuda", generator=g)], dim=1)
+    draft = torch.from_numpy(np.random.default_rng(5).integers(0, V, size=(B, K)).astype(np.int32)).cuda()
+    ws = aligned_workspace(dm.domino_verify_sample_workspace_bytes(B, K, V))
+    tau = torch.zeros(B, dtype=torch.int32, device="cuda")
+    tok = torch.zeros(B, dtype=torch.int32, device="cuda")
+    scrub = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    ts = []
+    for k in range(args.warmup + args.steps):
+        scrub.fill_(float(k))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dm.domino_verify_sample(dl, tl, draft, temperature=1.0, seed=k, tau_out=tau, token_out=tok, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+    if dm.domino_poll(ws) != 0:
+        raise RuntimeError("device error in verification")
+    t = statistics.mean(ts)
+    peaks, peak_kind = measured_peaks()
+    vbytes = (2 * K + 3) * B * V * 4
+    achieved = vbytes / t / 1e9
+    print(json.dumps({
+        "metric": "verified_blocks_per_s", "value": B / t, "unit": "blocks/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"speculative-sampling verification, {B} request(s), block {K}, V={V}, T=1",
+                   "l2": "flushed before every step"},
+        "roofline": {"kernel": "verify_sample (4 launches)", "bound": "hbm", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "algorithmic_bytes": vbytes, "peak_source": peak_kind},
+        "mean_tau": float(tau.float().mean().item()),
+    }), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -509,8 +565,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--batch", type=int, default=1, help="requests per GPU per draft block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["draft", "loss"], default="draft",
-                    help="draft: the draft block (default); loss: the teacher-forced training forward")
+    ap.add_argument("--mode", choices=["draft", "loss", "verify"], default="draft",
+                    help="draft: the draft block (default); loss: the teacher-forced training forward; "
+                         "verify: stochastic verification")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -518,6 +575,8 @@ def main(argv=None):
         run_reference(args)
     elif args.mode == "loss":
         run_loss(args)
+    elif args.mode == "verify":
+        run_verify(args)
     else:
         run_ours(args)
     _, _, world = dist_env()

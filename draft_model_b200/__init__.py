@@ -11,7 +11,7 @@ from ._binding import (DominoError, DominoWeights, STATUS, domino_correct_loop, 
                        domino_draft_block_events, domino_draft_block_host, domino_draft_loss,
                        domino_draft_loss_workspace_bytes, domino_launches_per_block, domino_lm_head, domino_poll,
                        domino_selftest_wait_timeout, domino_set_wait_budget_ns, domino_status_str, domino_verify,
-                       domino_workspace_bytes, domino_workspace_bytes_host, domino_workspace_init, library_path,
+                       domino_verify_sample, domino_verify_sample_workspace_bytes, domino_workspace_bytes, domino_workspace_bytes_host, domino_workspace_init, library_path,
                        load_library)
 
 GREEDY = 0
@@ -25,6 +25,6 @@ __all__ = [
     "domino_curriculum_loss_workspace_bytes", "domino_draft_block", "domino_draft_block_events",
     "domino_draft_block_host", "domino_draft_loss", "domino_draft_loss_workspace_bytes", "domino_launches_per_block",
     "domino_lm_head", "domino_poll", "domino_selftest_wait_timeout", "domino_set_wait_budget_ns", "domino_status_str",
-    "domino_verify", "domino_workspace_bytes", "domino_workspace_bytes_host", "domino_workspace_init",
+    "domino_verify", "domino_verify_sample", "domino_verify_sample_workspace_bytes", "domino_workspace_bytes", "domino_workspace_bytes_host", "domino_workspace_init",
     "library_path", "load_library",
 ]

@@ -54,6 +54,8 @@ def load_library() -> ctypes.CDLL:
         "domino_curriculum_loss": (I32, [P, P, P, I32, I32, I32, F, F, P, P, P, SZ, P]),
         "domino_draft_loss_workspace_bytes": (SZ, [W, I32, I32]),
         "domino_draft_loss": (I32, [W, P, P, P, I32, I32, F, F, P, P, P, SZ, P]),
+        "domino_verify_sample_workspace_bytes": (SZ, [I32, I32, I32]),
+        "domino_verify_sample": (I32, [P, P, P, I32, I32, I32, F, U64, P, P, P, SZ, P]),
         "domino_workspace_init": (I32, [P, SZ, P]),
         "domino_draft_block": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
         "domino_draft_block_events": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P,
@@ -231,6 +233,20 @@ def domino_draft_loss(w: DominoWeights, hidden, anchor, labels, *, lam: float, g
     _check(load_library().domino_draft_loss(w.ref, _ptr(hidden), _ptr(anchor), _ptr(labels), B, K, lam, gamma,
                                             _ptr(ce_out), _ptr(loss_out), wp, wn, _stream(stream)),
            "domino_draft_loss")
+
+
+def domino_verify_sample_workspace_bytes(B: int, K: int, V: int) -> int:
+    return int(load_library().domino_verify_sample_workspace_bytes(B, K, V))
+
+
+def domino_verify_sample(draft_logits, target_logits, draft, *, temperature: float, seed: int, tau_out, token_out,
+                         workspace, stream=None) -> None:
+    """Speculative sampling of a block: accepted draft tokens and the emitted token per request."""
+    B, K, V = draft_logits.shape
+    wp, wn = _ws(workspace)
+    _check(load_library().domino_verify_sample(_ptr(draft_logits), _ptr(target_logits), _ptr(draft), B, K, V,
+                                               temperature, seed, _ptr(tau_out), _ptr(token_out), wp, wn,
+                                               _stream(stream)), "domino_verify_sample")
 
 
 def domino_verify(draft, target, tau_out, stream=None) -> None:

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libdomino.so")
-SOURCES = ["domino_api.cu", "correct_loop.cu", "lm_head_tc.cu", "lm_head_f32.cu", "verify.cu", "noalloc.cu", "loop_tc.cu", "loss.cu"]
+SOURCES = ["domino_api.cu", "correct_loop.cu", "lm_head_tc.cu", "lm_head_f32.cu", "verify.cu", "noalloc.cu", "loop_tc.cu", "loss.cu", "verify_sample.cu"]
 HEADERS = ["common.cuh", "domino_internal.h", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -388,6 +388,29 @@ domino_status domino_draft_loss(const domino_weights* w, const void* hidden, con
                                                   ce_out, loss_out, reinterpret_cast<Control*>(ws + L.ctl), st));
 }
 
+size_t domino_verify_sample_workspace_bytes(int32_t B, int32_t K, int32_t V) {
+  if (B < 1 || K < 1 || K > 32 || V < 1) return 0;
+  return kCtlRegion + align_up(domino::verify_sample_scratch_bytes(B, K, V));
+}
+
+domino_status domino_verify_sample(const float* draft_logits, const float* target_logits, const int32_t* draft,
+                                   int32_t B, int32_t K, int32_t V, float temperature, uint64_t seed,
+                                   int32_t* tau_out, int32_t* token_out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (B < 1 || K < 1 || K > 32 || V < 1 || static_cast<long long>(B) * (2 * K + 1) > 65535) return DOMINO_ERR_INVALID_ARG;
+  if (!draft_logits || !target_logits || !draft || !tau_out || !token_out) return DOMINO_ERR_INVALID_ARG;
+  if (!aligned16(draft_logits) || !aligned16(target_logits) || !aligned16(draft) || !aligned16(tau_out) ||
+      !aligned16(token_out))
+    return DOMINO_ERR_INVALID_ARG;
+  if (!(temperature > 0.f && std::isfinite(temperature))) return DOMINO_ERR_INVALID_ARG;
+  domino_status s = check_workspace(workspace, workspace_bytes, domino_verify_sample_workspace_bytes(B, K, V));
+  if (s != DOMINO_OK) return s;
+  char* ws = static_cast<char*>(workspace);
+  return from_cuda(domino::launch_verify_sample(draft_logits, target_logits, draft, B, K, V, temperature, seed,
+                                                ws + kCtlRegion, tau_out, token_out, reinterpret_cast<Control*>(ws),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K, int32_t* tau_out,
                             void* stream) {
   if (!draft || !target || !tau_out || B < 1 || K < 1 || K > 32) return DOMINO_ERR_INVALID_ARG;

@@ -132,11 +132,20 @@ cudaError_t launch_lm_head_f32(const float* w, const float* hidden, float* out, 
 
 // Verification (stage 3).
 // Base-anchored curriculum loss over fp32 logit rows (loss.cu).
-int loss_chunks(int B, int K, int V);
+int lse_chunks(int rows, int V);
+cudaError_t launch_row_lse_partial(const float* X0, int K0, const float* X1, int K1, int B, int V, float scale,
+                                   int chunks, const int32_t* idx, int Kidx, float2* part, float* picked, Control* ctl,
+                                   cudaStream_t stream);
 size_t loss_scratch_bytes(int B, int K, int V);
 cudaError_t launch_curriculum_loss(const float* final_logits, const float* base_logits, const int32_t* labels, int B,
                                    int K, int V, float lambda, float gamma, void* scratch, float* ce_out,
                                    float* loss_out, Control* ctl, cudaStream_t stream);
+
+// Stochastic verification at T > 0 (verify_sample.cu).
+size_t verify_sample_scratch_bytes(int B, int K, int V);
+cudaError_t launch_verify_sample(const float* draft_logits, const float* target_logits, const int32_t* draft, int B,
+                                 int K, int V, float temperature, uint64_t seed, void* scratch, int32_t* tau_out,
+                                 int32_t* token_out, Control* ctl, cudaStream_t stream);
 
 cudaError_t launch_verify(const int32_t* draft, const int32_t* target, int B, int K, int32_t* tau,
                           cudaStream_t stream);

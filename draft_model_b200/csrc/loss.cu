@@ -9,9 +9,9 @@
 // positions and means over the batch.
 //
 // Two launches over rows of fp32 logits (R = B K rows per tensor, V columns):
-//   ce_partial_kernel  one CTA per (row, vocabulary chunk): coalesced pass with
-//                      an online (max, sum of exp) per thread, merged across the
-//                      CTA; the chunk holding the label also records its logit;
+//   row_lse_partial_kernel  one CTA per (row, vocabulary chunk): coalesced pass
+//                      with an online (max, sum of exp) per thread, merged across
+//                      the CTA; the chunk holding the label also records its logit;
 //   ce_combine_kernel  one CTA: log-sum-exp of every row from its chunks, the
 //                      row's cross-entropy, and the weighted loss, summed in fp64
 //                      in a fixed order (deterministic).
@@ -47,16 +47,25 @@ __device__ __forceinline__ void ms_push(MS& a, float x) {
   }
 }
 
-// blockIdx.y = row r in [0, 2R): tensor r / R (0 final, 1 base), row r % R;
-// blockIdx.x = vocabulary chunk.
-__global__ void __launch_bounds__(CE_THREADS) ce_partial_kernel(const float* __restrict__ final_logits,
-                                                                const float* __restrict__ base_logits, int R, int V,
-                                                                int chunks, const int32_t* __restrict__ labels,
-                                                                float2* __restrict__ part, float* __restrict__ picked,
-                                                                Control* ctl) {
+// Row log-sum-exp partials.  Rows r in [0, B (K0 + K1)): the B K0 rows of X0
+// (request b, position i at row b K0 + i), then the B K1 rows of X1.  CTA
+// (chunk c, row r) merges (max, sum exp(y - max)) of y = scale * x over the
+// row's c-th vocabulary chunk into part[r chunks + c]; the chunk holding
+// idx[b Kidx + i] (for i < Kidx, when idx is given) records that raw logit in
+// picked[r].  Out-of-range indices are clamped and flagged.
+__global__ void __launch_bounds__(CE_THREADS) row_lse_partial_kernel(const float* __restrict__ X0, int K0,
+                                                                     const float* __restrict__ X1, int K1, int B,
+                                                                     int V, float scale, int chunks,
+                                                                     const int32_t* __restrict__ idx, int Kidx,
+                                                                     float2* __restrict__ part,
+                                                                     float* __restrict__ picked, Control* ctl) {
   const int r = blockIdx.y, c = blockIdx.x;
-  const int rr = r % R;
-  const float* row = (r < R ? final_logits : base_logits) + static_cast<size_t>(rr) * V;
+  const int R0 = B * K0;
+  const bool first = r < R0;
+  const int rr = first ? r : r - R0;
+  const int Kr = first ? K0 : K1;
+  const int b = rr / Kr, i = rr % Kr;
+  const float* row = (first ? X0 : X1) + static_cast<size_t>(rr) * V;
   const int lo = static_cast<int>(static_cast<long long>(V) * c / chunks);
   const int hi = static_cast<int>(static_cast<long long>(V) * (c + 1) / chunks);
   MS a{-INFINITY, 0.f};
@@ -64,16 +73,16 @@ __global__ void __launch_bounds__(CE_THREADS) ce_partial_kernel(const float* __r
   for (; v + 3 * CE_THREADS < hi; v += 4 * CE_THREADS) {
     const float x0 = __ldcs(row + v), x1 = __ldcs(row + v + CE_THREADS);
     const float x2 = __ldcs(row + v + 2 * CE_THREADS), x3 = __ldcs(row + v + 3 * CE_THREADS);
-    ms_push(a, x0);
-    ms_push(a, x1);
-    ms_push(a, x2);
-    ms_push(a, x3);
+    ms_push(a, x0 * scale);
+    ms_push(a, x1 * scale);
+    ms_push(a, x2 * scale);
+    ms_push(a, x3 * scale);
   }
-  for (; v < hi; v += CE_THREADS) ms_push(a, __ldcs(row + v));
+  for (; v < hi; v += CE_THREADS) ms_push(a, __ldcs(row + v) * scale);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
-    const MS b{__shfl_xor_sync(0xFFFFFFFFu, a.m, o), __shfl_xor_sync(0xFFFFFFFFu, a.s, o)};
-    a = ms_merge(a, b);
+    const MS o2{__shfl_xor_sync(0xFFFFFFFFu, a.m, o), __shfl_xor_sync(0xFFFFFFFFu, a.s, o)};
+    a = ms_merge(a, o2);
   }
   __shared__ MS warp_ms[CE_THREADS / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -83,12 +92,14 @@ __global__ void __launch_bounds__(CE_THREADS) ce_partial_kernel(const float* __r
     MS t = warp_ms[0];
     for (int w = 1; w < CE_THREADS / 32; ++w) t = ms_merge(t, warp_ms[w]);
     part[static_cast<size_t>(r) * chunks + c] = make_float2(t.m, t.s);
-    int y = labels[rr];
-    if (y < 0 || y >= V) {
-      if (c == 0 && r < R) raise_error(ctl, ERRBIT_BAD_TOKEN);
-      y = min(max(y, 0), V - 1);
+    if (idx && i < Kidx) {
+      int y = idx[static_cast<size_t>(b) * Kidx + i];
+      if (y < 0 || y >= V) {
+        if (c == 0 && first) raise_error(ctl, ERRBIT_BAD_TOKEN);
+        y = min(max(y, 0), V - 1);
+      }
+      if (y >= lo && y < hi) picked[r] = row[y];
     }
-    if (y >= lo && y < hi) picked[r] = row[y];
   }
 }
 
@@ -108,7 +119,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS) ce_combine_kernel(const float
       for (int c = 0; c < chunks; ++c) M = fmaxf(M, p[c].x);
       double S = 0.0;
       for (int c = 0; c < chunks; ++c)
-        if (p[c].x != -INFINITY) S += static_cast<double>(p[c].y) * exp(static_cast<double>(p[c].x) - M);
+        if (p[c].x != -INFINITY) S += static_cast<double>(p[c].y * expf(p[c].x - M));
       ce[t] = static_cast<double>(M) + log(S) - static_cast<double>(picked[r]);
       if (ce_out) ce_out[static_cast<size_t>(rr) * 2 + t] = static_cast<float>(ce[t]);
     }
@@ -130,9 +141,8 @@ __global__ void __launch_bounds__(COMBINE_THREADS) ce_combine_kernel(const float
 
 }  // namespace
 
-int loss_chunks(int B, int K, int V) {
-  // about 1024 CTAs over the 2 B K rows, chunks of at least 2048 logits, at most 64
-  const int rows = 2 * B * K;
+int lse_chunks(int rows, int V) {
+  // about 1024 CTAs over the rows, chunks of at least 2048 logits, at most 64
   int c = (1024 + rows - 1) / rows;
   const int cap = V / 2048 > 0 ? V / 2048 : 1;
   if (c > cap) c = cap;
@@ -143,19 +153,27 @@ int loss_chunks(int B, int K, int V) {
 size_t loss_scratch_bytes(int B, int K, int V) {
   const size_t rows = 2ull * B * K;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  return al(rows * loss_chunks(B, K, V) * sizeof(float2)) + al(rows * sizeof(float));
+  return al(rows * lse_chunks(static_cast<int>(rows), V) * sizeof(float2)) + al(rows * sizeof(float));
+}
+
+cudaError_t launch_row_lse_partial(const float* X0, int K0, const float* X1, int K1, int B, int V, float scale,
+                                   int chunks, const int32_t* idx, int Kidx, float2* part, float* picked, Control* ctl,
+                                   cudaStream_t stream) {
+  row_lse_partial_kernel<<<dim3(chunks, B * (K0 + K1)), CE_THREADS, 0, stream>>>(X0, K0, X1, K1, B, V, scale, chunks,
+                                                                                 idx, Kidx, part, picked, ctl);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_curriculum_loss(const float* final_logits, const float* base_logits, const int32_t* labels, int B,
                                    int K, int V, float lambda, float gamma, void* scratch, float* ce_out,
                                    float* loss_out, Control* ctl, cudaStream_t stream) {
   const int R = B * K;
-  const int chunks = loss_chunks(B, K, V);
+  const int chunks = lse_chunks(2 * R, V);
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   float2* part = static_cast<float2*>(scratch);
   float* picked = reinterpret_cast<float*>(static_cast<char*>(scratch) + al(2ull * R * chunks * sizeof(float2)));
-  ce_partial_kernel<<<dim3(chunks, 2 * R), CE_THREADS, 0, stream>>>(final_logits, base_logits, R, V, chunks, labels,
-                                                                    part, picked, ctl);
+  row_lse_partial_kernel<<<dim3(chunks, 2 * R), CE_THREADS, 0, stream>>>(final_logits, K, base_logits, K, B, V, 1.f,
+                                                                         chunks, labels, K, part, picked, ctl);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ce_combine_kernel<<<1, COMBINE_THREADS, 0, stream>>>(part, picked, R, K, chunks, lambda, gamma, ce_out, loss_out);

@@ -217,6 +217,33 @@ DOMINO_API domino_status domino_draft_loss(const domino_weights* w, const void* 
                                            float* ce_out, float* loss_out, void* workspace,
                                            size_t workspace_bytes, void* stream);
 
+/* ---- Stochastic verification at T > 0 ----
+ * The pages report acceptance at T = 1 (study notes §三.2(1)) but give no
+ * mechanism; this is standard lossless speculative sampling.  With
+ * p_i = softmax(draft_logits[b, i, :] / T) (the final logits L_i the drafted
+ * tokens were sampled from, e.g. domino_draft_block's logits_out in GUMBEL mode)
+ * and q_i = softmax(target_logits[b, i, :] / T):
+ *   for i = 1..K: accept draft[b, i-1] with probability min(1, q_i(t) / p_i(t));
+ *   at the first rejection emit a token drawn from norm(max(0, q_i - p_i));
+ *   after K acceptances emit a bonus token drawn from q_{K+1}.
+ *   draft_logits  [B, K, V] fp32 device; target_logits [B, K+1, V] fp32 device
+ *   draft         [B, K] int32: the drafted tokens (out of range: clamped, flagged)
+ *   temperature   > 0; seed: Philox4x32-10 key (seed low, seed high); acceptance
+ *                 uniforms use counter (0, i-1, b, 2) word 0, the resampling
+ *                 Gumbel noise counter (j >> 2, i-1, b, 1) word j & 3 (streams
+ *                 the draft's Gumbel picks never use)
+ *   tau_out       [B] int32: accepted draft tokens (0..K)
+ *   token_out     [B] int32: the emitted residual or bonus token
+ *   workspace     domino_verify_sample_workspace_bytes(B, K, V) bytes, 256-byte
+ *                 aligned, zeroed once with domino_workspace_init.
+ * Four launches and one memset; asynchronous.  Argument errors (NULL,
+ * misaligned, T <= 0, K outside 1..32, B (2K+1) > 65535) return synchronously. */
+DOMINO_API size_t domino_verify_sample_workspace_bytes(int32_t B, int32_t K, int32_t V);
+DOMINO_API domino_status domino_verify_sample(const float* draft_logits, const float* target_logits,
+                                              const int32_t* draft, int32_t B, int32_t K, int32_t V,
+                                              float temperature, uint64_t seed, int32_t* tau_out, int32_t* token_out,
+                                              void* workspace, size_t workspace_bytes, void* stream);
+
 DOMINO_API domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K,
                             int32_t* tau_out, void* stream);
 

@@ -138,3 +138,16 @@ def test_loss_validation_is_host_side(lib):
     w = _cw()
     assert lib.domino_draft_loss_workspace_bytes(ctypes.byref(w), 1, 16) > lib.domino_workspace_bytes(ctypes.byref(w), 1, 16)
     assert lib.domino_draft_loss(ctypes.byref(w), p, p, None, 1, 16, 0.5, 1.0, None, p, p, 1 << 40, None) == INVALID
+
+
+def test_verify_sample_validation_is_host_side(lib):
+    INVALID = 1
+    p = 0x100000
+    n = lib.domino_verify_sample_workspace_bytes(2, 4, 1000)
+    assert n > 0 and lib.domino_verify_sample_workspace_bytes(2, 33, 1000) == 0
+    call = lambda T, B=2, K=4, draft=p: lib.domino_verify_sample(p, p, draft, B, K, 1000, T, 0, p, p, p, n, None)
+    assert call(0.0) == INVALID
+    assert call(float("nan")) == INVALID
+    assert call(1.0, K=0) == INVALID
+    assert call(1.0, B=2000, K=32) == INVALID
+    assert call(1.0, draft=None) == INVALID

@@ -1,0 +1,115 @@
+"""GPU parity of stochastic verification (speculative sampling) through the C ABI
+against oracle/sampling.py.
+
+Floating point decides integers here (accept or reject; the Gumbel-max draw), so
+the comparison follows the draft's protocol: a request whose acceptance test
+at any examined position lies within 1e-5 of its threshold (|u - q/p|) is a
+precision tie and only checked for validity; otherwise tau must match exactly,
+and the emitted token must score within 1e-3 of the oracle's best draw (it is
+the oracle's own pick wherever the oracle's top-2 margin exceeds that).
+"""
+import numpy as np
+import pytest
+import torch
+
+import draft_model_b200 as dm
+import oracle
+from _harness import aligned_workspace
+
+pytestmark = pytest.mark.gpu
+cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+ACCEPT_TIE = 1e-5
+SCORE_TIE = 1e-3
+
+
+def _gpu(dl, tl, draft, T, seed):
+    B, K, V = dl.shape
+    ws = aligned_workspace(dm.domino_verify_sample_workspace_bytes(B, K, V))
+    tau = torch.zeros(B, dtype=torch.int32, device="cuda")
+    tok = torch.zeros(B, dtype=torch.int32, device="cuda")
+    dm.domino_verify_sample(torch.from_numpy(dl).cuda(), torch.from_numpy(tl).cuda(), torch.from_numpy(draft).cuda(),
+                            temperature=T, seed=seed, tau_out=tau, token_out=tok, workspace=ws)
+    return tau.cpu().numpy(), tok.cpu().numpy(), dm.domino_poll(ws)
+
+
+def _oracle_scores(dl, tl, b, pos, T, seed):
+    K, V = dl.shape[1], dl.shape[2]
+    q = oracle.softmax_rows(tl[b, pos].astype(np.float64), T)
+    with np.errstate(divide="ignore"):
+        if pos < K:
+            p = oracle.softmax_rows(dl[b, pos].astype(np.float64), T)
+            return np.log(np.maximum(q - p, 0.0)) + oracle.resample_noise(seed, b, pos, V)
+        return np.log(q) + oracle.resample_noise(seed, b, K, V)
+
+
+def _check(dl, tl, draft, T, seed):
+    tau, tok, status = _gpu(dl, tl, draft, T, seed)
+    assert status == 0
+    ref = oracle.verify_sample(dl.astype(np.float64), tl.astype(np.float64), draft, T, seed)
+    B, K, V = dl.shape
+    stats = {"compared": 0, "ties": 0, "rejected": 0}
+    for b in range(B):
+        assert 0 <= tau[b] <= K and 0 <= tok[b] < V
+        examined = min(int(ref.tau[b]) + 1, K)
+        margin = np.abs(ref.uniform[b, :examined] - np.minimum(1.0, ref.ratio[b, :examined]))
+        if (margin < ACCEPT_TIE).any():
+            stats["ties"] += 1
+            continue
+        assert tau[b] == ref.tau[b], (b, tau[b], ref.tau[b])
+        score = _oracle_scores(dl, tl, b, int(ref.tau[b]), T, seed)
+        assert np.isfinite(score[tok[b]]), (b, tok[b])
+        assert score[tok[b]] >= score.max() - SCORE_TIE, (b, tok[b], int(np.argmax(score)))
+        stats["compared"] += 1
+        stats["rejected"] += int(ref.tau[b] < K)
+    return stats
+
+
+def _inputs(B, K, V, noise, seed):
+    rng = np.random.default_rng(seed)
+    dl = rng.normal(0.0, 2.0, size=(B, K, V)).astype(np.float32)
+    tl = np.concatenate([dl + rng.normal(0.0, noise, size=(B, K, V)), rng.normal(0.0, 2.0, size=(B, 1, V))],
+                        axis=1).astype(np.float32)
+    # drafted tokens: Gumbel-max samples of the draft distributions (any valid tokens would do)
+    g = -np.log(-np.log(rng.random(size=(B, K, V))))
+    draft = np.argmax(dl / 1.0 + g, axis=2).astype(np.int32)
+    return dl, tl, draft
+
+
+@cuda
+@pytest.mark.parametrize("B,K,V,noise,T,seed", [(6, 6, 5000, 0.5, 1.0, 1), (9, 16, 4100, 1.0, 1.0, 2),
+                                                (3, 4, 777, 0.3, 0.7, 3), (2, 16, 151936, 0.5, 1.0, 4),
+                                                (1, 1, 13, 2.0, 1.0, 5)])
+def test_verify_sample_matches_oracle(B, K, V, noise, T, seed):
+    dl, tl, draft = _inputs(B, K, V, noise, seed)
+    stats = _check(dl, tl, draft, T, seed)
+    assert stats["compared"] >= B - 1
+
+
+@cuda
+def test_verify_sample_mixes_accepts_and_rejects():
+    dl, tl, draft = _inputs(64, 3, 3000, 0.5, 6)
+    stats = _check(dl, tl, draft, 1.0, 6)
+    assert stats["compared"] >= 60
+    assert 5 <= stats["rejected"] <= stats["compared"] - 5
+
+
+@cuda
+def test_equal_distributions_accept_all():
+    rng = np.random.default_rng(7)
+    B, K, V = 4, 5, 2000
+    dl = rng.normal(size=(B, K, V)).astype(np.float32)
+    tl = np.concatenate([dl, rng.normal(size=(B, 1, V)).astype(np.float32)], axis=1)
+    draft = rng.integers(0, V, size=(B, K)).astype(np.int32)
+    tau, tok, status = _gpu(dl, tl, draft, 1.0, 9)
+    assert status == 0
+    np.testing.assert_array_equal(tau, K)
+    _check(dl, tl, draft, 1.0, 9)
+
+
+@cuda
+def test_bad_draft_token_is_flagged():
+    dl = np.zeros((1, 2, 100), dtype=np.float32)
+    tl = np.zeros((1, 3, 100), dtype=np.float32)
+    _, _, status = _gpu(dl, tl, np.array([[5, 100]], dtype=np.int32), 1.0, 0)
+    assert status == 6   # DOMINO_ERR_BAD_TOKEN
