@@ -302,6 +302,12 @@ def run_ours(args):
     cfg = workload_config(B)
     w = synth.make_weights(cfg)
     dw = device_weights(w, dev)
+    if args.gate_table:
+        # variant: token -> gate table built once per weight set (not timed)
+        from _harness import aligned_workspace
+        table = torch.empty((cfg.V, 3 * cfg.H), dtype=torch.float32, device=dev)
+        dm.domino_build_gate_table(dw, table, workspace=aligned_workspace(1024))
+        dw.set_gate_table(table)
     first = rank * B
     hidden_np = synth.make_hidden(cfg, B, first)
     anchor_np = synth.make_anchor(cfg, B, first)
@@ -403,7 +409,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD.format(B=B), "global_batch": B * world, "block_size": cfg.K,
+        "config": {"workload": WORKLOAD.format(B=B) + (", token->gate table variant" if args.gate_table else ""),
+                   "global_batch": B * world, "block_size": cfg.K,
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "l2": "flushed before every step (512 MiB write, outside the step timing)"},
         "us_per_block": t_max / args.steps / B * 1e6,
@@ -565,6 +572,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--batch", type=int, default=1, help="requests per GPU per draft block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gate-table", action="store_true",
+                    help="variant: precomputed token->gate table (G = W_ih E + b_ih) in the batched loop")
     ap.add_argument("--mode", choices=["draft", "loss", "verify"], default="draft",
                     help="draft: the draft block (default); loss: the teacher-forced training forward; "
                          "verify: stochastic verification")

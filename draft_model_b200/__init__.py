@@ -6,7 +6,8 @@ point names: it only marshals torch tensors (device memory) and CUDA streams to
 plain pointers.  There is no CPU fallback: every call raises if the library is
 missing or returns an error.
 """
-from ._binding import (DominoError, DominoWeights, STATUS, domino_correct_loop, domino_correct_loop_noalloc,
+from ._binding import (DominoError, DominoWeights, STATUS, domino_build_gate_table, domino_correct_loop,
+                       domino_correct_loop_noalloc, domino_gate_table_bytes,
                        domino_curriculum_loss, domino_curriculum_loss_workspace_bytes, domino_draft_block,
                        domino_draft_block_events, domino_draft_block_host, domino_draft_loss,
                        domino_draft_loss_workspace_bytes, domino_launches_per_block, domino_lm_head, domino_poll,
@@ -20,7 +21,8 @@ BF16 = 0
 F32 = 1
 
 __all__ = [
-    "DominoError", "DominoWeights", "STATUS", "GREEDY", "GUMBEL", "BF16", "F32",
+    "DominoError", "DominoWeights", "STATUS", "GREEDY", "GUMBEL", "BF16", "F32", "domino_build_gate_table",
+    "domino_gate_table_bytes",
     "domino_correct_loop", "domino_correct_loop_noalloc", "domino_curriculum_loss",
     "domino_curriculum_loss_workspace_bytes", "domino_draft_block", "domino_draft_block_events",
     "domino_draft_block_host", "domino_draft_loss", "domino_draft_loss_workspace_bytes", "domino_launches_per_block",

@@ -28,7 +28,7 @@ class _CWeights(ctypes.Structure):
         ("gru_hidden", ctypes.c_int32), ("rank", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("w_lm", ctypes.c_void_p), ("embed", ctypes.c_void_p), ("w_ih", ctypes.c_void_p),
         ("w_hh", ctypes.c_void_p), ("b_ih", ctypes.c_void_p), ("b_hh", ctypes.c_void_p),
-        ("w1", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+        ("w1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("gate_table", ctypes.c_void_p),
     ]
 
 
@@ -55,6 +55,8 @@ def load_library() -> ctypes.CDLL:
         "domino_draft_loss_workspace_bytes": (SZ, [W, I32, I32]),
         "domino_draft_loss": (I32, [W, P, P, P, I32, I32, F, F, P, P, P, SZ, P]),
         "domino_verify_sample_workspace_bytes": (SZ, [I32, I32, I32]),
+        "domino_gate_table_bytes": (SZ, [W]),
+        "domino_build_gate_table": (I32, [W, P, P, SZ, P]),
         "domino_verify_sample": (I32, [P, P, P, I32, I32, I32, F, U64, P, P, P, SZ, P]),
         "domino_workspace_init": (I32, [P, SZ, P]),
         "domino_draft_block": (I32, [W, P, P, I32, I32, I32, F, U64, P, P, P, P, P, P, SZ, P]),
@@ -132,6 +134,11 @@ class DominoWeights:
     @property
     def ref(self):
         return ctypes.byref(self.c)
+
+    def set_gate_table(self, table) -> None:
+        """Use a [V, 3H] float32 token->gate table (domino_build_gate_table), or None."""
+        self.gate_table = table
+        self.c.gate_table = _ptr(table)
 
 
 # ---------------------------------------------------------------- entry points (same names as the C ABI)
@@ -247,6 +254,17 @@ def domino_verify_sample(draft_logits, target_logits, draft, *, temperature: flo
     _check(load_library().domino_verify_sample(_ptr(draft_logits), _ptr(target_logits), _ptr(draft), B, K, V,
                                                temperature, seed, _ptr(tau_out), _ptr(token_out), wp, wn,
                                                _stream(stream)), "domino_verify_sample")
+
+
+def domino_gate_table_bytes(w: DominoWeights) -> int:
+    return int(load_library().domino_gate_table_bytes(w.ref))
+
+
+def domino_build_gate_table(w: DominoWeights, table_out, *, workspace, stream=None) -> None:
+    """G[t] = W_ih E[t] + b_ih for every token into a [V, 3H] float32 tensor."""
+    wp, wn = _ws(workspace)
+    _check(load_library().domino_build_gate_table(w.ref, _ptr(table_out), wp, wn, _stream(stream)),
+           "domino_build_gate_table")
 
 
 def domino_verify(draft, target, tau_out, stream=None) -> None:

@@ -153,7 +153,9 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
     t.gi_part = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(domino::kLoopTcMaxSplits) * B * 3 * H * 4);
     t.gh_part = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(domino::kLoopTcMaxSplits) * B * 3 * H * 4);
     t.u_part = reinterpret_cast<float*>(p); p += al(static_cast<size_t>(domino::kLoopTcMaxSplits) * B * r * 4);
-    t.U2 = reinterpret_cast<__nv_bfloat16*>(p);
+    t.U2 = reinterpret_cast<__nv_bfloat16*>(p); p += al(static_cast<size_t>(2) * B * r * 2);
+    t.fed = reinterpret_cast<int32_t*>(p);
+    t.gate_table = w->gate_table;
     t.best = reinterpret_cast<unsigned long long*>(ws + L.best);
     t.ctl = reinterpret_cast<Control*>(ws + L.ctl);
     t.budget_ns = g_budget_ns.load();
@@ -246,7 +248,9 @@ int32_t domino_launches_per_block(const domino_weights* w, int32_t B, int32_t K)
   if (!weights_ok(w) || B < 1 || K < 1 || K > 32) return -1;
   if (use_loop_tc(w, B)) {
     const int chunks = (B + domino::kLoopTcReqPerLaunch - 1) / domino::kLoopTcReqPerLaunch;
-    return 1 /* LM head */ + 1 /* anchor embeddings */ + K * (domino::kLoopTcLaunchesPerStep + chunks);
+    // with a token->gate table the first position needs no gate GEMM (W_hh S = 0)
+    return 1 /* LM head */ + 1 /* anchor tokens */ + K * (domino::kLoopTcLaunchesPerStep + chunks) -
+           (w->gate_table ? 1 : 0);
   }
   const int NB = domino::loop_group_size(B);
   return 1 /* LM head */ + (B + NB - 1) / NB;
@@ -325,6 +329,37 @@ domino_status domino_draft_block(const domino_weights* w, const void* hidden, co
                                  void* workspace, size_t workspace_bytes, void* stream) {
   return domino_draft_block_events(w, hidden, anchor, B, K, mode, temperature, seed, forced, target, draft_out,
                                    logits_out, tau_out, workspace, workspace_bytes, stream, nullptr);
+}
+
+// ---------------------------------------------------------------- token -> gate table
+
+size_t domino_gate_table_bytes(const domino_weights* w) {
+  if (!weights_ok(w)) return 0;
+  return static_cast<size_t>(w->vocab) * 3 * w->gru_hidden * 4;
+}
+
+domino_status domino_build_gate_table(const domino_weights* w, float* table_out, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!weights_ok(w) || !table_out || !aligned16(table_out)) return DOMINO_ERR_INVALID_ARG;
+  if (!w->embed || !aligned16(w->embed) || !w->w_ih || !aligned16(w->w_ih)) return DOMINO_ERR_INVALID_ARG;
+  if (w->b_ih && !aligned16(w->b_ih)) return DOMINO_ERR_INVALID_ARG;
+  domino_status s = check_workspace(workspace, workspace_bytes, kCtlRegion);
+  if (s != DOMINO_OK) return s;
+  const int sms = num_sms();
+  if (sms <= 0) return DOMINO_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G3 = 3 * w->gru_hidden;
+  cudaError_t e;
+  // G[t, :] = W_ih E[t, :] for every token: the LM-head GEMM with the embedding
+  // rows as its positions and W_ih as its row operand (output [V, 3H])
+  if (w->dtype == DOMINO_BF16)
+    e = domino::launch_lm_head_tc(w->w_ih, w->embed, table_out, G3, w->vocab, w->embed_dim, nullptr, 0, 0, nullptr,
+                                  nullptr, nullptr, static_cast<Control*>(workspace), g_budget_ns.load(), sms, st);
+  else
+    e = domino::launch_lm_head_f32(static_cast<const float*>(w->w_ih), static_cast<const float*>(w->embed), table_out,
+                                   G3, w->vocab, w->embed_dim, w->embed_dim, st);
+  if (e == cudaSuccess && w->b_ih) e = domino::launch_add_row_bias(table_out, w->b_ih, w->vocab, G3, sms, st);
+  return from_cuda(e);
 }
 
 // ---------------------------------------------------------------- training forward

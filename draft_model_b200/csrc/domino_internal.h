@@ -94,12 +94,16 @@ struct LoopTcArgs {
   float* u_part;           // [kLoopTcMaxSplits, B, r]
   __nv_bfloat16* U2;       // [2B, r]  interleaved bf16 hi / lo rows of u
   unsigned long long* best;  // [K, B]
+  int32_t* fed;            // [B]     token fed to the GRU after the current position
+  const float* gate_table; // [V, 3H] token->gate table E W_ih^T + b_ih, or null
   Control* ctl;
   uint64_t budget_ns, seed;
   float temperature;
   int mode, B, K, V, d, E, H, r, num_sms;
 };
 cudaError_t run_loop_tc(const LoopTcArgs& args, cudaStream_t stream);
+cudaError_t launch_add_row_bias(float* table, const float* bias, size_t rows, int cols, int num_sms,
+                                cudaStream_t stream);
 // Shapes the tensor-core path accepts (16-byte aligned tensor-map strides, < 2^16 vocabulary tiles).
 bool loop_tc_supported(int E, int H, int d, int r, int V);
 // H rounded up to whole 64-wide k-blocks: each bf16 half of S2 has this many columns.
@@ -110,7 +114,8 @@ inline size_t loop_tc_scratch_bytes(int B, int E, int H, int r) {
   const size_t Hp = static_cast<size_t>(loop_tc_padded_h(H));
   return al(static_cast<size_t>(B) * E * 2) + al(static_cast<size_t>(B) * H * 4) + al(static_cast<size_t>(B) * 2 * Hp * 2) +
          2 * al(static_cast<size_t>(kLoopTcMaxSplits) * B * 3 * H * 4) +
-         al(static_cast<size_t>(kLoopTcMaxSplits) * B * r * 4) + al(static_cast<size_t>(2) * B * r * 2);
+         al(static_cast<size_t>(kLoopTcMaxSplits) * B * r * 4) + al(static_cast<size_t>(2) * B * r * 2) +
+         al(static_cast<size_t>(B) * 4);
 }
 
 // LM head (stage 1).

@@ -390,11 +390,14 @@ __global__ void __launch_bounds__(NTH, 1)
 // GRU for every (request, unit): sums the split-K partials, applies the gates,
 // keeps S (fp32) and writes its bf16 hi / lo halves (row stride 2*Hp) for the
 // next tensor-core products.
+// With a token->gate table, gi is the fed token's table row (b_ih included)
+// instead of the W_ih X partials.
 __global__ void __launch_bounds__(256) gru_step_kernel(const float* __restrict__ gi_part, int gi_splits,
                                                        const float* __restrict__ gh_part, int gh_splits,
                                                        const float* __restrict__ b_ih, const float* __restrict__ b_hh,
-                                                       float* __restrict__ S, __nv_bfloat16* __restrict__ S2, int B,
-                                                       int H, int Hp) {
+                                                       const float* __restrict__ table,
+                                                       const int32_t* __restrict__ fed, float* __restrict__ S,
+                                                       __nv_bfloat16* __restrict__ S2, int B, int H, int Hp) {
   griddep_launch_dependents();
   griddep_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -406,9 +409,14 @@ __global__ void __launch_bounds__(256) gru_step_kernel(const float* __restrict__
 #pragma unroll
   for (int g = 0; g < 3; ++g) {
     const size_t at = static_cast<size_t>(b) * G3 + static_cast<size_t>(g) * H + j;
-    float si = b_ih ? b_ih[g * H + j] : 0.f, sh = b_hh ? b_hh[g * H + j] : 0.f;
+    float si, sh = b_hh ? b_hh[g * H + j] : 0.f;
+    if (table) {
+      si = table[static_cast<size_t>(fed[b]) * G3 + static_cast<size_t>(g) * H + j];
+    } else {
+      si = b_ih ? b_ih[g * H + j] : 0.f;
 #pragma unroll 4
-    for (int s = 0; s < gi_splits; ++s) si += gi_part[s * gstride + at];
+      for (int s = 0; s < gi_splits; ++s) si += gi_part[s * gstride + at];
+    }
 #pragma unroll 4
     for (int s = 0; s < gh_splits; ++s) sh += gh_part[s * gstride + at];
     gi[g] = si;
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(256) pick_step_kernel(unsigned long long* best
                                                         const int32_t* __restrict__ forced,
                                                         const int32_t* __restrict__ target, int32_t* draft,
                                                         int32_t* tau, const __nv_bfloat16* __restrict__ embed,
-                                                        __nv_bfloat16* X, Control* ctl) {
+                                                        __nv_bfloat16* X, int32_t* fed_out, Control* ctl) {
   // one block per request: thread 0 decides the token, all threads copy the row
   griddep_launch_dependents();
   griddep_wait();
@@ -479,9 +487,10 @@ __global__ void __launch_bounds__(256) pick_step_kernel(unsigned long long* best
       f = min(max(f, 0), V - 1);
     }
     fed = f;
+    fed_out[b] = f;
   }
   __syncthreads();
-  if (step + 1 >= K) return;
+  if (step + 1 >= K || X == nullptr) return;   // no embedding rows with a token->gate table
   const uint4* src = reinterpret_cast<const uint4*>(embed + static_cast<size_t>(fed) * E);
   uint4* dst = reinterpret_cast<uint4*>(X + static_cast<size_t>(b) * E);
   for (int q = threadIdx.x; q < E / 8; q += blockDim.x) dst[q] = __ldg(src + q);
@@ -538,7 +547,21 @@ int splits_for(int num_sms, int tiles, int num_kb) {
   return clampi(num_sms / (tiles > 0 ? tiles : 1), 1, cap);
 }
 
+// table[t, c] += bias[c] over a [rows, cols] fp32 table
+__global__ void add_row_bias_kernel(float* __restrict__ table, const float* __restrict__ bias, size_t rows, int cols) {
+  const size_t n = rows * static_cast<size_t>(cols);
+  for (size_t q = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; q < n;
+       q += static_cast<size_t>(gridDim.x) * blockDim.x)
+    table[q] += bias[q % cols];
+}
+
 }  // namespace
+
+cudaError_t launch_add_row_bias(float* table, const float* bias, size_t rows, int cols, int num_sms,
+                                cudaStream_t stream) {
+  add_row_bias_kernel<<<num_sms * 4, 256, 0, stream>>>(table, bias, rows, cols);
+  return cudaGetLastError();
+}
 
 bool loop_tc_supported(int E, int H, int d, int r, int V) {
   // every tensor map row stride and the W1 state-column base must be 16-byte
@@ -585,6 +608,13 @@ cudaError_t run_loop_tc(const LoopTcArgs& L, cudaStream_t st) {
   Prob& p1 = g.p[1];
   p1.nrows = G3; p1.M = B; p1.num_vt = vt; p1.num_mt = num_mt; p1.num_kb = kb1; p1.splits = s1; p1.a_kwrap = Hp;
   p1.out = L.gh_part; p1.split_stride = static_cast<size_t>(B) * G3;
+  // W_hh S alone (token->gate table): split to about one unit per SM
+  GArgs gh = g;
+  gh.nprob = 1;
+  gh.p[0] = p1;
+  const int sh1 = splits_for(L.num_sms, vt * num_mt, kb1);
+  gh.p[0].splits = sh1;
+  gh.units0 = gh.units = vt * num_mt * sh1;
 
   // ---- bottleneck GEMM: W1_s (r x H) against S' hi | lo
   GArgs bk = g;
@@ -601,21 +631,30 @@ cudaError_t run_loop_tc(const LoopTcArgs& L, cudaStream_t st) {
   if ((e = cudaMemsetAsync(L.S, 0, static_cast<size_t>(B) * H * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(L.S2, 0, static_cast<size_t>(B) * 2 * Hp * 2, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(L.best, 0, static_cast<size_t>(K) * B * 8, st)) != cudaSuccess) return e;
+  __nv_bfloat16* Xg = L.gate_table ? nullptr : L.X;   // fed embeddings only when W_ih multiplies them
   e = launch_pdl(pick_step_kernel, dim3(B), dim3(256), 0, st, L.best, -1, K, B, V, E, L.anchor, L.forced, L.target,
-                 L.draft, L.tau, static_cast<const __nv_bfloat16*>(L.embed), L.X, L.ctl);
+                 L.draft, L.tau, static_cast<const __nv_bfloat16*>(L.embed), Xg, L.fed, L.ctl);
   if (e != cudaSuccess) return e;
 
   for (int i = 0; i < K; ++i) {
-    // 1. gate GEMMs (W_hh S is zero at the first position: S = 0)
-    g.nprob = i == 0 ? 1 : 2;
-    g.units0 = vt * num_mt * s0;
-    g.units = g.units0 + (i == 0 ? 0 : vt * num_mt * s1);
-    const int grid0 = g.units < L.num_sms ? g.units : L.num_sms;
-    e = launch_pdl(gemm_tc_kernel<EPI_PARTIAL>, dim3(grid0), dim3(NTH), gsm, st, tWih, tX, tWhh, tS2, g);
-    if (e != cudaSuccess) return e;
+    // 1. gate GEMMs (W_hh S is zero at the first position: S = 0); with a
+    //    token->gate table only W_hh S is multiplied
+    if (!L.gate_table) {
+      g.nprob = i == 0 ? 1 : 2;
+      g.units0 = vt * num_mt * s0;
+      g.units = g.units0 + (i == 0 ? 0 : vt * num_mt * s1);
+      const int grid0 = g.units < L.num_sms ? g.units : L.num_sms;
+      e = launch_pdl(gemm_tc_kernel<EPI_PARTIAL>, dim3(grid0), dim3(NTH), gsm, st, tWih, tX, tWhh, tS2, g);
+      if (e != cudaSuccess) return e;
+    } else if (i > 0) {
+      const int gridh = gh.units < L.num_sms ? gh.units : L.num_sms;
+      e = launch_pdl(gemm_tc_kernel<EPI_PARTIAL>, dim3(gridh), dim3(NTH), gsm, st, tWhh, tS2, tWhh, tS2, gh);
+      if (e != cudaSuccess) return e;
+    }
     // 2. GRU
     e = launch_pdl(gru_step_kernel, dim3((B * H + 255) / 256), dim3(256), 0, st, L.gi_part, s0, L.gh_part,
-                   i == 0 ? 0 : s1, L.b_ih, L.b_hh, L.S, L.S2, B, H, Hp);
+                   i == 0 ? 0 : (L.gate_table ? sh1 : s1), L.b_ih, L.b_hh, L.gate_table,
+                   static_cast<const int32_t*>(L.fed), L.S, L.S2, B, H, Hp);
     if (e != cudaSuccess) return e;
     // 3. bottleneck product, 4. SiLU and the hi / lo split of u
     e = launch_pdl(gemm_tc_kernel<EPI_PARTIAL>, dim3(gridb), dim3(NTH), gsm, st, tW1s, tS2, tW1s, tS2, bk);
@@ -652,7 +691,7 @@ cudaError_t run_loop_tc(const LoopTcArgs& L, cudaStream_t st) {
     }
     // 6. picks, next fed tokens and embeddings (verification after the last position)
     e = launch_pdl(pick_step_kernel, dim3(B), dim3(256), 0, st, L.best, i, K, B, V, E, L.anchor, L.forced, L.target,
-                   L.draft, L.tau, static_cast<const __nv_bfloat16*>(L.embed), L.X, L.ctl);
+                   L.draft, L.tau, static_cast<const __nv_bfloat16*>(L.embed), Xg, L.fed, L.ctl);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

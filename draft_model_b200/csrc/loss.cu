@@ -70,13 +70,13 @@ __global__ void __launch_bounds__(CE_THREADS) row_lse_partial_kernel(const float
   const int hi = static_cast<int>(static_cast<long long>(V) * (c + 1) / chunks);
   MS a{-INFINITY, 0.f};
   int v = lo + static_cast<int>(threadIdx.x);
-  for (; v + 3 * CE_THREADS < hi; v += 4 * CE_THREADS) {
-    const float x0 = __ldcs(row + v), x1 = __ldcs(row + v + CE_THREADS);
-    const float x2 = __ldcs(row + v + 2 * CE_THREADS), x3 = __ldcs(row + v + 3 * CE_THREADS);
-    ms_push(a, x0 * scale);
-    ms_push(a, x1 * scale);
-    ms_push(a, x2 * scale);
-    ms_push(a, x3 * scale);
+  // eight independent loads in flight per thread (about 56 KB per SM with seven CTAs)
+  for (; v + 7 * CE_THREADS < hi; v += 8 * CE_THREADS) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = __ldcs(row + v + u * CE_THREADS);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) ms_push(a, x[u] * scale);
   }
   for (; v < hi; v += CE_THREADS) ms_push(a, __ldcs(row + v) * scale);
 #pragma unroll

@@ -91,6 +91,12 @@ typedef struct {
   const void* w1;      /* [r, d + H] bottleneck; columns [0, d) act on h_i,        */
                        /* columns [d, d + H) on the GRU state S_{i-1}               */
   const void* w2;      /* [V, r]   vocabulary projection of the correction         */
+  const float* gate_table; /* [V, 3H] f32 token -> gate table G[t] = W_ih E[t] + b_ih  */
+                       /* (domino_build_gate_table), or NULL.  When set, the       */
+                       /* batched (tensor-core) loop reads the fed token's row      */
+                       /* instead of multiplying W_ih; the persistent loop (small   */
+                       /* batches, fp32) ignores it.  Not from the pages: an        */
+                       /* inference-time restructuring of the GRU's input side.     */
 } domino_weights;
 
 /* Workspace bytes needed by domino_draft_block / domino_lm_head /
@@ -178,6 +184,18 @@ DOMINO_API domino_status domino_correct_loop_noalloc(const domino_weights* w, co
                                           int32_t* tau_out, void* stream);
 
 /* Stage 3 only: tau_out[b] = number of leading i with draft[b, i] == target[b, i]. */
+/* ---- Token -> gate table ----
+ * G[t, :] = W_ih E[t, :] + b_ih for every token t (fp32, [V, 3H] row-major,
+ * domino_gate_table_bytes(w) bytes), computed once per weight set: the GRU's
+ * input-side pre-activation depends on the fed token only, so a loop given the
+ * table (domino_weights.gate_table) gathers one 3H row per request per position
+ * instead of streaming W_ih.  bf16 weights: one tcgen05 GEMM launch (fp32
+ * accumulation, as in the loop) plus a bias launch; fp32: SIMT.  workspace:
+ * at least 1024 bytes, 256-byte aligned, zeroed once (error word).  Asynchronous. */
+DOMINO_API size_t domino_gate_table_bytes(const domino_weights* w);
+DOMINO_API domino_status domino_build_gate_table(const domino_weights* w, float* table_out, void* workspace,
+                                                 size_t workspace_bytes, void* stream);
+
 /* ---- Training forward (Domino study notes, gsyq.cn, §二.2 配套专属训练方案) ----
  *
  * Base-anchored curriculum loss (§二.2(2)) on given logits:

@@ -151,3 +151,16 @@ def test_verify_sample_validation_is_host_side(lib):
     assert call(1.0, K=0) == INVALID
     assert call(1.0, B=2000, K=32) == INVALID
     assert call(1.0, draft=None) == INVALID
+
+
+def test_gate_table_abi(lib):
+    w = _cw(V=1000, H=64)
+    assert lib.domino_gate_table_bytes(ctypes.byref(w)) == 1000 * 3 * 64 * 4
+    assert lib.domino_gate_table_bytes(ctypes.byref(_cw(d=4095))) == 0
+    # NULL or misaligned table: rejected before any CUDA call
+    assert lib.domino_build_gate_table(ctypes.byref(w), None, 0x100000, 1024, None) == 1
+    assert lib.domino_build_gate_table(ctypes.byref(w), 0x100004, 0x100000, 1024, None) == 1
+    # a table changes the batched loop's launch count by one (no gate GEMM at the first position)
+    n0 = lib.domino_launches_per_block(ctypes.byref(w), 8, 16)
+    w.gate_table = 0x200000
+    assert lib.domino_launches_per_block(ctypes.byref(w), 8, 16) == n0 - 1
