@@ -187,7 +187,7 @@ __device__ __forceinline__ Sched make_sched(const LoopArgs& a, int c, int G) {
   s.p = partition_of(a, c, G);
   s.e3 = Seg{a.nsegE3, a.segE3};
   s.h3 = Seg{a.nsegH3, a.segH3};
-  s.nIH = (s.p.j1 - s.p.j0) * s.e3.n;
+  s.nIH = a.gate_table ? 0 : (s.p.j1 - s.p.j0) * s.e3.n;   // a token->gate table replaces the W_ih items
   s.nHH = (s.p.j1 - s.p.j0) * s.h3.n;
   s.nC = (s.p.v1 - s.p.v0 + VCHUNK - 1) / VCHUNK;
   s.per_step = s.nIH + s.nC + s.nHH;
@@ -455,7 +455,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
     sh.fed[tid] = t;
   }
   named_barrier(BAR_CONS, CONS_THREADS);
-  gather_rows<W, CONS_THREADS>(a, sh, NB);
+  if (!a.gate_table) gather_rows<W, CONS_THREADS>(a, sh, NB);
   grid_arrive<CONS_THREADS>(a, sh);         // zeroed keys and accumulators visible to all
   grid_wait<CONS_THREADS>(a, sh, nbar++);
 
@@ -497,8 +497,14 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
           gi[g] = sh.bias[jl * 6 + g];
           gh[g] = sh.bias[jl * 6 + 3 + g];
         }
-        for (int s = 0; s < sc.e3.n; ++s)
-          for (int g = 0; g < 3; ++g) gi[g] += sh.part_ih[(jl * sc.e3.n + s) * 32 + g * NB + b];
+        if (a.gate_table) {
+          // the fed token's row of G = W_ih E + b_ih (sh.fed is always a valid token)
+          const float* trow = a.gate_table + static_cast<size_t>(sh.fed[b]) * 3 * a.H;
+          for (int g = 0; g < 3; ++g) gi[g] = trow[g * a.H + j];
+        } else {
+          for (int s = 0; s < sc.e3.n; ++s)
+            for (int g = 0; g < 3; ++g) gi[g] += sh.part_ih[(jl * sc.e3.n + s) * 32 + g * NB + b];
+        }
         for (int s = 0; s < sc.h3.n; ++s)
           for (int g = 0; g < 3; ++g) gh[g] += sh.part_hh[(jl * sc.h3.n + s) * 32 + g * NB + b];
         const float r = sigmoid_fast(gi[0] + gh[0]);
@@ -668,7 +674,7 @@ __device__ void consumer(const LoopArgs& a, const Shared& sh, const Sched& sc) {
       sh.fed[b] = f;
     }
     named_barrier(BAR_CONS, CONS_THREADS);
-    if (i + 1 < K && !aborted(sh)) gather_rows<W, CONS_THREADS>(a, sh, nb);
+    if (i + 1 < K && !aborted(sh) && !a.gate_table) gather_rows<W, CONS_THREADS>(a, sh, nb);
     named_barrier(BAR_CONS, CONS_THREADS);
   }
 

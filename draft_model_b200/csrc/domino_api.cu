@@ -175,6 +175,7 @@ domino_status run_loop(const domino_weights* w, const void* hidden, const float*
   a.b_hh = w->b_hh;
   a.w1 = w->w1;
   a.w2 = w->w2;
+  a.gate_table = w->gate_table;
   a.ctl = reinterpret_cast<Control*>(ws + L.ctl);
   a.S_glob = reinterpret_cast<float*>(ws + L.S);
   a.u_acc = reinterpret_cast<long long*>(ws + L.u);

@@ -30,6 +30,7 @@ struct LoopArgs {
   const float* b_hh;
   const void* w1;
   const void* w2;
+  const float* gate_table;  // [V, 3H] token->gate table W_ih E + b_ih, or null (then W_ih is streamed)
   // inputs (already offset to the group's first request)
   const void* hidden;   // [nb, K, d]
   const float* base;    // [nb, K, V]

@@ -93,10 +93,10 @@ typedef struct {
   const void* w2;      /* [V, r]   vocabulary projection of the correction         */
   const float* gate_table; /* [V, 3H] f32 token -> gate table G[t] = W_ih E[t] + b_ih  */
                        /* (domino_build_gate_table), or NULL.  When set, the       */
-                       /* batched (tensor-core) loop reads the fed token's row      */
-                       /* instead of multiplying W_ih; the persistent loop (small   */
-                       /* batches, fp32) ignores it.  Not from the pages: an        */
-                       /* inference-time restructuring of the GRU's input side.     */
+                       /* correction loop reads the fed token's row instead of     */
+                       /* multiplying W_ih (domino_correct_loop_noalloc ignores    */
+                       /* it).  Not from the pages: an inference-time              */
+                       /* restructuring of the GRU's input side.                   */
 } domino_weights;
 
 /* Workspace bytes needed by domino_draft_block / domino_lm_head /

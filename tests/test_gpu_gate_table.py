@@ -60,19 +60,36 @@ def test_gate_table_full_size_sampled_rows():
 
 
 @cuda
-@pytest.mark.parametrize("cfg", [_small(), _small(B=17, K=5, mode="gumbel", temperature=1.0, seed=8)],
-                         ids=["greedy_b9", "gumbel_b17"])
+@pytest.mark.parametrize("cfg", [_small(), _small(B=17, K=5, mode="gumbel", temperature=1.0, seed=8),
+                                 _small(B=1, K=16, seed=10), _small(B=3, K=8, mode="gumbel", temperature=0.8, seed=11),
+                                 synth.CONFIGS["tiny_f32"]],
+                         ids=["greedy_b9", "gumbel_b17", "persistent_b1", "persistent_gumbel_b3", "tiny_f32"])
 def test_block_with_gate_table(cfg):
     w = synth.make_weights(cfg)
     m = oracle.Model.from_storage(w)
     dw = device_weights(w)
+    n0 = dm.domino_launches_per_block(dw, cfg.B, cfg.K)
     dw.set_gate_table(_table(dw))
-    assert dm.domino_launches_per_block(dw, cfg.B, cfg.K) == 2 + cfg.K * 6 - 1
+    # the batched loop drops the first position's gate GEMM; the persistent loop's count is unchanged
+    assert dm.domino_launches_per_block(dw, cfg.B, cfg.K) == (n0 - 1 if cfg.B >= 4 and cfg.dtype == "bf16" else n0)
     hidden, anchor = synth.make_hidden(cfg), synth.make_anchor(cfg)
     gpu = run_gpu(dw, cfg, hidden, anchor)
     assert gpu["status"] == 0
     _, stats = check_against_oracle(m, cfg, hidden, anchor, gpu)
     assert stats["agree"] > 0.5
+
+
+@cuda
+def test_block_with_gate_table_full_size_b1():
+    cfg = synth.CONFIGS["qwen3_8b_b1"]
+    w = synth.make_weights(cfg)
+    m = oracle.Model.from_storage(w)
+    dw = device_weights(w)
+    dw.set_gate_table(_table(dw))
+    hidden, anchor = synth.make_hidden(cfg), synth.make_anchor(cfg)
+    gpu = run_gpu(dw, cfg, hidden, anchor)
+    assert gpu["status"] == 0
+    check_against_oracle(m, cfg, hidden, anchor, gpu)
 
 
 @cuda
