@@ -94,20 +94,17 @@ __device__ __forceinline__ SegIter seg_begin(const TcArgs& a, int ntiles) {
   return it;
 }
 
-// Tile t -> (operand, vocabulary tile, position tile).  The second A operand's
-// tiles come first so they never land in the stream-K tail.  W_lm tiles run with
-// the position tile slowest: CTAs on different position tiles then stream the
-// same W_lm rows at about the same time, and the repeats are L2 hits.
-__device__ __forceinline__ void tile_decode(const TcArgs& a, int ntiles2, int t, bool& second, int& vt, int& mt) {
-  second = t < ntiles2;
-  if (second) {
-    vt = t / a.num_mt;
-    mt = t % a.num_mt;
-  } else {
-    const int tt = t - ntiles2;
-    mt = tt / a.num_vt;
-    vt = tt % a.num_vt;
-  }
+// Tile t -> (operand, vocabulary tile, position tile).  Tiles run position tile
+// by position tile, each block being the W_lm tiles and then the second A
+// operand's tiles of that position tile: with the k-stages split evenly over
+// the CTAs, the CTAs on different position tiles then stream the same W_lm rows
+// at about the same time, and the repeats are L2 hits.
+__device__ __forceinline__ void tile_decode(const TcArgs& a, int t, bool& second, int& vt, int& mt) {
+  const int per_mt = a.num_vt + a.num_vt2;
+  mt = t / per_mt;
+  const int rem = t % per_mt;
+  second = rem >= a.num_vt;
+  vt = second ? rem - a.num_vt : rem;
 }
 
 __global__ void __launch_bounds__(NTH, 1)
@@ -129,9 +126,7 @@ __global__ void __launch_bounds__(NTH, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // tiles of the second A operand come first so they never land in the tail
-  const int ntiles2 = a.num_vt2 * a.num_mt;
-  const int ntiles = ntiles2 + a.num_vt * a.num_mt;
+  const int ntiles = (a.num_vt + a.num_vt2) * a.num_mt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -182,7 +177,7 @@ __global__ void __launch_bounds__(NTH, 1)
       while (ok && si.next(a, ntiles, g)) {
         bool second;
         int vt, mt;
-        tile_decode(a, ntiles2, g.t, second, vt, mt);
+        tile_decode(a, g.t, second, vt, mt);
         const CUtensorMap* tA = second ? &tmA2 : &tmA;
         for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
           if (it >= a.stages && !bounded_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
@@ -259,7 +254,7 @@ __global__ void __launch_bounds__(NTH, 1)
       tc_fence_after();
       bool second;
       int vt, mt;
-      tile_decode(a, ntiles2, g.t, second, vt, mt);
+      tile_decode(a, g.t, second, vt, mt);
       const int row = q * 32 + lane;                 // row of the 128-row tile
       const int v = vt * BM + row;
       const int nrows = second ? a.rows2 : a.V;
