@@ -36,6 +36,9 @@
 //   ---- barrier arrive; meanwhile W_hh S_i partial dots for step i+1 (ring);
 //        barrier wait -> picks, next embedding rows
 // Delta L and L_i never touch HBM unless final logits are requested.
+// With a token->gate table (LoopArgs::gate_table, G = W_ih E + b_ih built once per
+// weight set) the W_ih items are dropped from the ring, the GRU epilogue reads
+// the fed token's row of G, and no embedding rows are gathered.
 #include <cstdint>
 
 #include "common.cuh"
