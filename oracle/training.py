@@ -17,7 +17,7 @@ What it computes, from the Domino study notes (gsyq.cn), §二.2 配套专属训
    and every position's loss carrying an exponentially decaying weight that
    favours the front of the block.
 
-Readings where the notes are silent (listed in the design doc):
+Readings where the notes are silent:
 - the per-position loss is the cross-entropy -log softmax(L)[y] of the logits
   without temperature;
 - the decay weight of block position i+1 (i = 0..K-1) is w_i = gamma**i with
