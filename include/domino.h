@@ -11,6 +11,9 @@
  *      picked and fed back (study notes §二.1(2); yhxrc.cn §四);
  *   3. greedy verification against target tokens, giving the acceptance length
  *      tau (study notes §一.1; digest page "大三本科生一作…" §4).
+ * Beside the block: the teacher-forced training forward with its base-anchored
+ * curriculum loss (study notes §二.2), stochastic verification at T > 0, and a
+ * precomputed token->gate table for the GRU's input side (see below).
  *
  * Conventions shared by every entry point
  *   - Tensor pointers are DEVICE pointers owned by the caller, except where an
@@ -57,8 +60,9 @@ typedef enum {
                                /* for the co-resident correction grid)                   */
   DOMINO_ERR_CUDA = 4,         /* a CUDA runtime call failed                             */
   DOMINO_ERR_TIMEOUT = 5,      /* a bounded device wait ran out of time (device-side)    */
-  DOMINO_ERR_BAD_TOKEN = 6,    /* an anchor or forced token was outside [0, V); it was   */
-                               /* clamped and the block still ran (device-side)          */
+  DOMINO_ERR_BAD_TOKEN = 6,    /* an anchor, forced, label or drafted token was outside  */
+                               /* [0, V); it was clamped and the work still ran          */
+                               /* (device-side)                                          */
   DOMINO_ERR_WORKSPACE = 7     /* workspace missing, too small or misaligned             */
 } domino_status;
 
@@ -183,7 +187,6 @@ DOMINO_API domino_status domino_correct_loop_noalloc(const domino_weights* w, co
                                           const int32_t* target, int32_t* draft_out, float* logits_out,
                                           int32_t* tau_out, void* stream);
 
-/* Stage 3 only: tau_out[b] = number of leading i with draft[b, i] == target[b, i]. */
 /* ---- Token -> gate table ----
  * G[t, :] = W_ih E[t, :] + b_ih for every token t (fp32, [V, 3H] row-major,
  * domino_gate_table_bytes(w) bytes), computed once per weight set: the GRU's
@@ -262,6 +265,7 @@ DOMINO_API domino_status domino_verify_sample(const float* draft_logits, const f
                                               float temperature, uint64_t seed, int32_t* tau_out, int32_t* token_out,
                                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Stage 3 only: tau_out[b] = number of leading i with draft[b, i] == target[b, i]. */
 DOMINO_API domino_status domino_verify(const int32_t* draft, const int32_t* target, int32_t B, int32_t K,
                             int32_t* tau_out, void* stream);
 
