@@ -236,3 +236,41 @@ def test_full_size_sweep_b256_sampled():
     gpu = run_gpu(dw, cfg, hidden, anchor, want_logits=False)
     assert gpu["status"] == 0
     check_against_oracle(m, cfg, hidden, anchor, gpu, rows=[0, 100, 255])
+
+
+# ---------------------------------------------------------------- degenerate cases
+
+@cuda
+@pytest.mark.parametrize("cfg", [small(B=1, K=1, seed=21), small(B=6, K=1, seed=22),
+                                 small(B=5, K=1, mode="gumbel", temperature=1.0, seed=23)],
+                         ids=["persistent", "tensor_core", "gumbel_tc"])
+def test_single_position_block(cfg):
+    w, m, dw = setup(cfg)
+    hidden, anchor = synth.make_hidden(cfg), synth.make_anchor(cfg)
+    target = np.zeros((cfg.B, 1), dtype=np.int32)
+    gpu = run_gpu(dw, cfg, hidden, anchor, target=target)
+    assert gpu["status"] == 0
+    check_against_oracle(m, cfg, hidden, anchor, gpu, target=target)
+
+
+@cuda
+@pytest.mark.parametrize("B", [2, 6], ids=["persistent", "tensor_core"])
+def test_exact_ties_pick_the_lowest_index(B):
+    # W2 = 0 (L_i = L_base) and a dominant W_lm row copied to several tokens: their
+    # base logits are bit-identical maxima, and the pick must be the lowest of them
+    cfg = small(B=B, K=4, seed=24)
+    w = synth.make_weights(cfg)
+    w.w2 = np.zeros_like(w.w2)
+    hidden = synth.make_hidden(cfg)
+    h0 = oracle.widen_f64(hidden, "bf16")[0, 0]
+    row = synth.f32_to_bf16_bits((np.sign(h0) * 0.5).astype(np.float32))
+    tied = [4097, 137, 2500, 4999]
+    w.w_lm = w.w_lm.copy()
+    for t in tied:
+        w.w_lm[t] = row
+    dw = device_weights(w)
+    hidden[:, :, :] = hidden[0, 0]          # every position sees the same hidden state
+    anchor = synth.make_anchor(cfg)
+    gpu = run_gpu(dw, cfg, hidden, anchor)
+    assert gpu["status"] == 0
+    np.testing.assert_array_equal(gpu["tokens"], min(tied))
