@@ -386,7 +386,8 @@ def run_ours(args):
     peaks, peak_kind = measured_peaks()
     lbytes = loop_bytes(cfg, B)
     achieved = lbytes / loop_avg / 1e9
-    traffic = recorded_traffic("correct_loop_kernel") if B == 1 else None
+    # recorded for the standard B=1 loop only (the gate-table variant reads no W_ih)
+    traffic = recorded_traffic("correct_loop_kernel") if B == 1 and not args.gate_table else None
     lm_frac_hbm = lm_head_bytes(cfg, B) / lm_avg / 1e9 / peaks["hbm_gbs"]
     lm_tflops = lm_head_flops(cfg, B) / lm_avg / 1e12
     # the LM head runs inside a long back-to-back step: the sustained (power-capped)
