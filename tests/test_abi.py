@@ -164,3 +164,31 @@ def test_gate_table_abi(lib):
     n0 = lib.domino_launches_per_block(ctypes.byref(w), 8, 16)
     w.gate_table = 0x200000
     assert lib.domino_launches_per_block(ctypes.byref(w), 8, 16) == n0 - 1
+
+
+def test_stage_entry_points_validate_on_the_host(lib):
+    INVALID, UNSUP, WS = 1, 2, 7
+    w = _cw()
+    p, ws, big = 0x100000, 0x200000, 1 << 40
+    # stage 1
+    assert lib.domino_lm_head(ctypes.byref(w), p, 0, 16, p, ws, big, None) == INVALID
+    assert lib.domino_lm_head(ctypes.byref(w), None, 1, 16, p, ws, big, None) == INVALID
+    assert lib.domino_lm_head(ctypes.byref(w), p, 1, 16, 0x100008, ws, big, None) == INVALID   # misaligned out
+    assert lib.domino_lm_head(ctypes.byref(w), p, 1, 16, p, None, big, None) == WS
+    # stage 2 with given base logits
+    loop = lambda B=1, K=16, base=p, ws_=ws: lib.domino_correct_loop(ctypes.byref(w), p, base, p, B, K, 0, 1.0, 0,
+                                                                     None, None, p, None, None, ws_, big, None)
+    assert loop(K=33) == INVALID
+    assert loop(base=None) == INVALID
+    assert loop(ws_=0x200010) == WS
+    # host-buffer entry point
+    assert lib.domino_draft_block_host(ctypes.byref(w), None, p, 1, 16, 0, 1.0, 0, None, None, p, None, ws, big,
+                                       None) == INVALID
+    assert lib.domino_draft_block_host(ctypes.byref(w), p, p, 1, 16, 0, 1.0, 0, None, p, p, None, ws, big,
+                                       None) == INVALID                     # target without tau
+    # allocation-free loop: its fixed scratch limits are checked before any device work
+    noalloc = lambda B=1, K=16, ww=w: lib.domino_correct_loop_noalloc(ctypes.byref(ww), p, p, p, B, K, 0, 1.0, 0,
+                                                                      None, None, p, None, None, None)
+    assert noalloc(B=9) == UNSUP
+    assert noalloc(ww=_cw(H=8192)) == UNSUP
+    assert noalloc(K=0) == INVALID
