@@ -297,6 +297,31 @@ def test_first_position_sees_anchor_step_hand_computed():
     np.testing.assert_allclose(res.logits[0, 0], want, rtol=0, atol=1e-15)
 
 
+def test_first_position_reads_each_requests_anchor_embedding_hand_computed():
+    """The GRU's first input is E[anchor] of that request (H = E = d = r = 1).
+
+    Only W_ih, the embedding and W2 are nonzero, so S_1 = (1 - z) n with
+    r = sigmoid(W_ir x), z = sigmoid(W_iz x), n = tanh(W_in x), x = E[anchor],
+    and L_1 = W2 SiLU(S_1).  Anchor 0 has a zero embedding, so feeding any
+    token but the anchor changes the logits.
+    """
+    V = 3
+    emb = np.array([[0.0], [0.5], [-1.5]], np.float32)
+    w_ih = np.array([[0.4], [-0.3], [0.8]], np.float32)
+    w = synth.Weights(
+        dtype="f32", w_lm=np.zeros((V, 1), np.float32), embed=emb, w_ih=w_ih,
+        w_hh=np.zeros((3, 1), np.float32), b_ih=None, b_hh=None,
+        w1=np.array([[0.0, 1.0]], np.float32), w2=np.array([[1.0], [2.0], [-1.0]], np.float32))
+    res = draft_block(Model.from_storage(w), np.zeros((2, 1, 1), np.float32), np.array([2, 1]))
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))  # noqa: E731
+    for b, anchor in enumerate((2, 1)):
+        x = float(emb[anchor, 0])
+        z = sig(float(w_ih[1, 0]) * x)
+        s1 = (1.0 - z) * math.tanh(float(w_ih[2, 0]) * x)
+        u = s1 * sig(s1)
+        np.testing.assert_allclose(res.logits[b, 0], [u, 2.0 * u, -u], rtol=0, atol=1e-15)
+
+
 def test_bruteforce_greedy_fixed_point():
     cfg = small_cfg(B=1, K=3, V=5, d=6, H=3, r=2, E=4, seed=5)
     w, m = model_of(cfg)

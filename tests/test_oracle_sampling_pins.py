@@ -1,9 +1,10 @@
 """Pins of the stochastic-verification oracle (oracle/sampling.py): the exact
-output law of speculative sampling, its acceptance probability, and its limits.
+output law of speculative sampling, its acceptance probability, the law of the
+acceptance length and of the residual draw, and its limits.
 CPU only."""
 import numpy as np
 import pytest
-from scipy import stats
+from scipy import special, stats
 
 from oracle import accept_uniform, resample_noise, softmax_rows, verify_sample
 
@@ -88,3 +89,55 @@ def test_deterministic_and_tau_range():
     np.testing.assert_array_equal(r1.tau, r2.tau)
     np.testing.assert_array_equal(r1.token, r2.token)
     assert ((r1.tau >= 0) & (r1.tau <= K)).all()
+
+
+@pytest.mark.parametrize("T", [0.5, 1.0, 2.5])
+def test_softmax_rows_matches_scipy_at_temperature(T):
+    x = np.random.default_rng(5).normal(0.0, 3.0, size=(4, 7, 33))
+    np.testing.assert_allclose(softmax_rows(x, T), special.softmax(x / T, axis=-1), rtol=1e-13, atol=0)
+
+
+def test_softmax_rows_temperature_limits():
+    x = np.array([[0.3, 1.9, -0.4, 1.2]])
+    cold = softmax_rows(x, 1e-3)                     # T -> 0: one-hot at the argmax
+    np.testing.assert_allclose(cold, [[0.0, 1.0, 0.0, 0.0]], atol=1e-12)
+    hot = softmax_rows(x, 1e6)                       # T -> inf: uniform
+    np.testing.assert_allclose(hot, 0.25, atol=1e-6)
+
+
+def test_acceptance_length_law_is_the_product_of_acceptances():
+    # with independent uniforms, P(tau >= k) = prod_{i <= k} a_i, a_i = min(1, q_i(t_i) / p_i(t_i))
+    K, T = 3, 1.0
+    want = np.array([0.7, 0.5, 0.6])                  # acceptance of token 0 at each position
+    pd = np.array([[0.5, 0.2, 0.2, 0.1]] * K)
+    qd = np.stack([[0.5 * x, 0.2, 0.3, 0.5 - 0.5 * x] for x in want])
+    dl, tl = np.log(pd)[None], np.log(np.concatenate([qd, [[0.25] * 4]]))[None]
+    p, q = softmax_rows(dl, T)[0], softmax_rows(tl, T)[0]
+    draft = np.zeros((1, K), dtype=np.int64)
+    a = np.array([min(1.0, q[i, 0] / p[i, 0]) for i in range(K)])
+    np.testing.assert_allclose(a, want, rtol=1e-12)
+    at_least = np.concatenate([[1.0], np.cumprod(a)])            # P(tau >= k), k = 0..K
+    law = at_least - np.concatenate([at_least[1:], [0.0]])       # P(tau == k)
+    n = 6000
+    counts = np.bincount([int(verify_sample(dl, tl, draft, T, seed=s).tau[0]) for s in range(n)], minlength=K + 1)
+    assert stats.chisquare(counts, law * n).pvalue > 1e-3, (counts / n, law)
+
+
+def test_residual_draw_follows_the_normalised_residual():
+    # given a rejection at position 1, the emitted token is distributed as norm(max(0, q_1 - p_1))
+    V, T = 4, 1.0
+    dl = np.log(np.array([[[0.10, 0.60, 0.15, 0.15]]]))
+    tl = np.log(np.array([[[0.30, 0.10, 0.30, 0.30], [0.25, 0.25, 0.25, 0.25]]]))
+    p, q = softmax_rows(dl, T)[0, 0], softmax_rows(tl, T)[0, 0]
+    resid = np.maximum(q - p, 0.0)
+    resid /= resid.sum()
+    draft = np.array([[1]])                           # a = q(1) / p(1) = 1/6
+    tokens = []
+    for s in range(12000):
+        res = verify_sample(dl, tl, draft, T, seed=s)
+        if res.tau[0] == 0:
+            tokens.append(int(res.token[0]))
+    counts = np.bincount(tokens, minlength=V)
+    assert counts[1] == 0                             # the rejected token has no residual mass
+    keep = resid > 0
+    assert stats.chisquare(counts[keep], resid[keep] * len(tokens)).pvalue > 1e-3, (counts / len(tokens), resid)
