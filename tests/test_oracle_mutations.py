@@ -60,6 +60,13 @@ MUTATIONS = [
     ("forced_tokens_ignored", "domino_ref.py",
      "prev = np.asarray(forced, dtype=np.int64)[:, p] if forced is not None else pick.astype(np.int64)",
      "prev = pick.astype(np.int64)", 1),
+    ("margin_sides_swapped", "domino_ref.py",
+     "        top2[:, p] = srt[:, 0]\n        top1[:, p] = srt[:, 1]",
+     "        top2[:, p] = srt[:, 1]\n        top1[:, p] = srt[:, 0]", 1),
+    ("forced_gap_sign", "domino_ref.py",
+     "gap[:, p] = top1[:, p] - score[np.arange(B), fed]", "gap[:, p] = score[np.arange(B), fed] - top1[:, p]", 1),
+    ("lm_head_rows_position_major", "domino_ref.py",
+     "hk = hidden64.reshape(B * K, d)", "hk = hidden64.transpose(1, 0, 2).reshape(B * K, d)", 1),
     ("gumbel_temperature_multiplies", "domino_ref.py", "score = L / temperature + g", "score = L * temperature + g", 1),
     ("gumbel_noise_shared_by_requests", "domino_ref.py",
      "gumbel_noise(seed, int(rid[b]), p + 1, V)", "gumbel_noise(seed, 0, p + 1, V)", 1),

@@ -9,9 +9,11 @@ wrong sign or index, a transposed operand, a swapped gate) fails at least one:
 * LM head           -> brute-force triple loop
 * correction        -> W2 = 0 and W1 = 0 reduce every pick to argmax of the base logits
 * [h ; S] order     -> zeroing either column block removes exactly that dependence
-* state indexing    -> position 1 already sees GRU(e(anchor), 0) (hand-computed)
+* state indexing    -> position 1 already sees GRU(e(anchor), 0) (hand-computed),
+                       with each request's own anchor embedding as that input
 * loop              -> teacher forcing on the free-running picks changes nothing;
                        causality; brute-force greedy fixed point
+* pick margins      -> top1 / top2 / forced_gap by sorting each position's scores
 * Gumbel-max        -> chi-square against the exact law prod_i softmax(L_i / T)[t_i];
                        noise moments (Euler-Mascheroni mean, pi^2/6 variance)
 * tau               -> brute force over every mismatch position
@@ -339,6 +341,32 @@ def test_bruteforce_greedy_fixed_point():
 
 
 # ---------------------------------------------------------------- tau / shapes / configs
+
+@pytest.mark.parametrize("mode", ["greedy", "gumbel"])
+def test_pick_margins_bruteforce(mode):
+    """top1 / top2 are the two largest pick scores and forced_gap = top1 - score(fed) >= 0.
+
+    The parity protocol accepts a GPU pick within a margin of the best, so these
+    fields are checked by sorting each position's scores directly.
+    """
+    cfg = small_cfg(B=3, K=5, V=40)
+    w, m = model_of(cfg)
+    hidden, anchor = synth.make_hidden(cfg), synth.make_anchor(cfg)
+    fed = np.random.default_rng(8).integers(0, cfg.V, size=(cfg.B, cfg.K))
+    T, seed = 0.8, 21
+    res = draft_block(m, hidden, anchor, forced=fed, mode=mode, temperature=T, seed=seed)
+    for b in range(cfg.B):
+        for p in range(cfg.K):
+            score = [float(x) for x in res.logits[b, p]]
+            if mode == "gumbel":
+                g = gumbel_noise(seed, b, p + 1, cfg.V)
+                score = [score[j] / T + float(g[j]) for j in range(cfg.V)]
+            order = sorted(range(cfg.V), key=lambda j: (-score[j], j))
+            assert res.tokens[b, p] == order[0]
+            assert res.top1[b, p] == score[order[0]] and res.top2[b, p] == score[order[1]]
+            assert res.forced_gap[b, p] == score[order[0]] - score[int(fed[b, p])]
+            assert res.forced_gap[b, p] >= 0.0
+
 
 def test_tau_bruteforce():
     rng = np.random.default_rng(4)
