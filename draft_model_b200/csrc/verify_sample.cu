@@ -16,7 +16,8 @@
 //   accept_kernel          one warp per request: the K acceptance tests in parallel;
 //   resample_kernel        CTA per (vocabulary chunk, request): Gumbel-max over
 //                          the residual (or the bonus row), 64-bit atomicMax;
-//   finish_kernel          tau and the emitted token.
+//   finish_kernel          warp per request: tau and the emitted token (a draw
+//                          from q when the residual had no positive fp32 entry).
 // HBM-bound: the draft and target rows are read once, plus one row pair again.
 #include <cmath>
 #include <cstdint>
@@ -126,12 +127,38 @@ __global__ void __launch_bounds__(256) resample_kernel(const float* __restrict__
   }
 }
 
-__global__ void finish_kernel(const unsigned long long* __restrict__ best, const int32_t* __restrict__ pos, int B,
-                              int32_t* __restrict__ tau_out, int32_t* __restrict__ token_out) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= B) return;
-  tau_out[b] = pos[b];
-  token_out[b] = static_cast<int32_t>(argmax_key_index(best[b]));
+// One warp per request: tau and the emitted token.  A rejection whose residual
+// max(0, q - p) had no positive entry in fp32 (p and q agree to working
+// precision except at the drafted token, whose probability lies below it) left
+// no key; the token is then drawn from q at that position with the same noise
+// (Gumbel-max over log q), which keeps the emitted token's law q.
+__global__ void __launch_bounds__(32) finish_kernel(const float* __restrict__ target_logits, int K, int V, float scale,
+                                                    uint64_t seed, const unsigned long long* __restrict__ best,
+                                                    const int32_t* __restrict__ pos_in,
+                                                    const double* __restrict__ lse_q_in,
+                                                    int32_t* __restrict__ tau_out, int32_t* __restrict__ token_out) {
+  const int b = blockIdx.x, lane = threadIdx.x;
+  const int pos = pos_in[b];
+  unsigned long long key = best[b];
+  if (key == 0ull) {   // warp-uniform
+    const float lse_q = static_cast<float>(lse_q_in[b]);
+    const float* rq = target_logits + (static_cast<size_t>(b) * (K + 1) + pos) * V;
+    for (int j = lane; j < V; j += 32) {
+      const float u = philox_uniform(seed, static_cast<uint32_t>(j) >> 2, static_cast<uint32_t>(pos),
+                                     static_cast<uint32_t>(b), kStreamResample, static_cast<uint32_t>(j) & 3u);
+      const unsigned long long k = argmax_key(rq[j] * scale - lse_q - logf(-logf(u)), static_cast<uint32_t>(j));
+      key = k > key ? k : key;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, key, o);
+      key = other > key ? other : key;
+    }
+  }
+  if (lane == 0) {
+    tau_out[b] = pos;
+    token_out[b] = static_cast<int32_t>(argmax_key_index(key));
+  }
 }
 
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -174,7 +201,7 @@ cudaError_t launch_verify_sample(const float* draft_logits, const float* target_
   resample_kernel<<<dim3(rchunks, B), 256, 0, stream>>>(draft_logits, target_logits, B, K, V, scale, rchunks, seed, pos,
                                                         lse_p, lse_q, best);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  finish_kernel<<<(B + 127) / 128, 128, 0, stream>>>(best, pos, B, tau_out, token_out);
+  finish_kernel<<<B, 32, 0, stream>>>(target_logits, K, V, scale, seed, best, pos, lse_q, tau_out, token_out);
   return cudaGetLastError();
 }
 

@@ -247,6 +247,9 @@ DOMINO_API domino_status domino_draft_loss(const domino_weights* w, const void* 
  *   for i = 1..K: accept draft[b, i-1] with probability min(1, q_i(t) / p_i(t));
  *   at the first rejection emit a token drawn from norm(max(0, q_i - p_i));
  *   after K acceptances emit a bonus token drawn from q_{K+1}.
+ * A rejection whose residual max(0, q_i - p_i) has no positive fp32 entry
+ * (p_i and q_i agree to working precision except at the drafted token, whose
+ * probability lies below it) emits a token drawn from q_i instead.
  *   draft_logits  [B, K, V] fp32 device; target_logits [B, K+1, V] fp32 device
  *   draft         [B, K] int32: the drafted tokens (out of range: clamped, flagged)
  *   temperature   > 0; seed: Philox4x32-10 key (seed low, seed high); acceptance

@@ -18,7 +18,7 @@ its acceptance rate, and its p == q and q(t) == 0 limits.
 """
 from .domino_ref import Model, Result, draft_block, gru_cell, lm_head, positions, sigmoid, silu, verify, widen_f64
 from .philox import gumbel_noise, philox4x32_10, philox4x32_10_np, uniform_from_word
-from .sampling import VerifyResult, accept_uniform, resample_noise, softmax_rows, verify_sample
+from .sampling import VerifyResult, accept_uniform, emission_scores, resample_noise, softmax_rows, verify_sample
 from .training import cross_entropy_rows, curriculum_loss, position_weights, train_forward
 
 __all__ = ["Model", "Result", "draft_block", "gru_cell", "lm_head", "positions", "sigmoid", "silu", "verify",

@@ -23,6 +23,12 @@ seed), on streams the draft never uses (counter word 3):
     bonus): Gumbel g[j] = -log(-log u) from counter (j >> 2, i - 1, b, 1),
     word j & 3; the residual sample is argmax_j (log r[j] + g[j]) (Gumbel-max,
     log 0 = -inf), the bonus argmax_j (log q[j] + g[j]).
+
+A degenerate case the rule leaves open: a rejection whose residual
+max(0, q_i - p_i) is zero everywhere in working precision.  This happens when
+p_i and q_i agree to that precision except at the drafted token, whose
+probability lies below it.  Reading taken here: the token is then drawn from
+q_i with the same noise, which keeps the law of the emitted token equal to q_i.
 """
 from __future__ import annotations
 
@@ -52,6 +58,23 @@ def resample_noise(seed: int, b: int, pos0: int, V: int) -> np.ndarray:
     """Gumbel noise over the vocabulary for the residual / bonus sample at 0-based position pos0."""
     u = uniform_from_word(_words(seed, b, pos0, STREAM_RESAMPLE, (V + 3) // 4)[:V])
     return -np.log(-np.log(u))
+
+
+def emission_scores(p_row, q_row, seed: int, b: int, pos0: int) -> np.ndarray:
+    """Gumbel-max scores of the token emitted after the accepted prefix of request b.
+
+    p_row is None for the bonus draw (pos0 = K): scores log q + g.  Otherwise
+    the residual draw at the rejected 0-based position pos0: log max(0, q - p) + g,
+    or log q + g when the residual is zero everywhere.
+    """
+    q_row = np.asarray(q_row, dtype=np.float64)
+    noise = resample_noise(seed, b, pos0, q_row.shape[-1])
+    with np.errstate(divide="ignore"):
+        if p_row is not None:
+            resid = np.maximum(q_row - np.asarray(p_row, dtype=np.float64), 0.0)
+            if (resid > 0.0).any():
+                return np.log(resid) + noise
+        return np.log(q_row) + noise
 
 
 def softmax_rows(logits: np.ndarray, temperature: float) -> np.ndarray:
@@ -95,12 +118,9 @@ def verify_sample(draft_logits: np.ndarray, target_logits: np.ndarray, draft: np
                 pos = i
                 break
         if pos < K:
-            resid = np.maximum(q[b, pos] - p[b, pos], 0.0)
-            with np.errstate(divide="ignore"):
-                score = np.log(resid) + resample_noise(seed, b, pos, V)
+            score = emission_scores(p[b, pos], q[b, pos], seed, b, pos)
         else:
-            with np.errstate(divide="ignore"):
-                score = np.log(q[b, K]) + resample_noise(seed, b, K, V)
+            score = emission_scores(None, q[b, K], seed, b, K)
         tau[b] = pos
         token[b] = int(np.argmax(score))
         srt = np.sort(score)[-2:]

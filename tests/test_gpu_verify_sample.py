@@ -34,13 +34,10 @@ def _gpu(dl, tl, draft, T, seed):
 
 
 def _oracle_scores(dl, tl, b, pos, T, seed):
-    K, V = dl.shape[1], dl.shape[2]
+    K = dl.shape[1]
     q = oracle.softmax_rows(tl[b, pos].astype(np.float64), T)
-    with np.errstate(divide="ignore"):
-        if pos < K:
-            p = oracle.softmax_rows(dl[b, pos].astype(np.float64), T)
-            return np.log(np.maximum(q - p, 0.0)) + oracle.resample_noise(seed, b, pos, V)
-        return np.log(q) + oracle.resample_noise(seed, b, K, V)
+    p = oracle.softmax_rows(dl[b, pos].astype(np.float64), T) if pos < K else None
+    return oracle.emission_scores(p, q, seed, b, pos)
 
 
 def _check(dl, tl, draft, T, seed):
@@ -113,3 +110,26 @@ def test_bad_draft_token_is_flagged():
     tl = np.zeros((1, 3, 100), dtype=np.float32)
     _, _, status = _gpu(dl, tl, np.array([[5, 100]], dtype=np.int32), 1.0, 0)
     assert status == 6   # DOMINO_ERR_BAD_TOKEN
+
+
+@cuda
+def test_empty_residual_draws_from_the_target():
+    # draft and target rows equal except the drafted token, whose probability
+    # (~e^-60) lies below fp32 and fp64 resolution: rejections (ratio e^-1) leave a
+    # residual with no positive entry on either side, and the token comes from q
+    rng = np.random.default_rng(12)
+    B, K, V = 48, 2, 3000
+    dl = rng.normal(0.0, 2.0, size=(B, K, V)).astype(np.float32)
+    draft = rng.integers(0, V, size=(B, K)).astype(np.int32)
+    dl[np.arange(B), 0, draft[:, 0]] = -60.0
+    tl = np.concatenate([dl, rng.normal(0.0, 2.0, size=(B, 1, V)).astype(np.float32)], axis=1)
+    tl[np.arange(B), 0, draft[:, 0]] = -61.0
+    stats = _check(dl, tl, draft, 1.0, 13)
+    assert stats["rejected"] >= 15
+    ref = oracle.verify_sample(dl.astype(np.float64), tl.astype(np.float64), draft, 1.0, 13)
+    tau, tok, _ = _gpu(dl, tl, draft, 1.0, 13)
+    assert ((tok >= 0) & (tok < V)).all()
+    for b in np.flatnonzero(ref.tau == 0):
+        q = oracle.softmax_rows(tl[b, 0].astype(np.float64), 1.0)
+        p = oracle.softmax_rows(dl[b, 0].astype(np.float64), 1.0)
+        assert not (np.maximum(q - p, 0.0) > 0).any()

@@ -96,10 +96,13 @@ MUTATIONS = [
     ("ratio_inverted", "sampling.py",
      "ratio[b, i] = q[b, i, t] / p[b, i, t]", "ratio[b, i] = p[b, i, t] / q[b, i, t]", 1),
     ("residual_sign", "sampling.py",
-     "np.maximum(q[b, pos] - p[b, pos], 0.0)", "np.maximum(p[b, pos] - q[b, pos], 0.0)", 1),
+     "np.maximum(q_row - np.asarray(p_row, dtype=np.float64), 0.0)",
+     "np.maximum(np.asarray(p_row, dtype=np.float64) - q_row, 0.0)", 1),
     ("resample_from_target_not_residual", "sampling.py",
-     "resid = np.maximum(q[b, pos] - p[b, pos], 0.0)", "resid = q[b, pos]", 1),
-    ("bonus_from_last_draft_position", "sampling.py", "np.log(q[b, K])", "np.log(q[b, K - 1])", 1),
+     "resid = np.maximum(q_row - np.asarray(p_row, dtype=np.float64), 0.0)", "resid = q_row", 1),
+    ("empty_residual_fallback_dropped", "sampling.py", "if (resid > 0.0).any():", "if True:", 1),
+    ("bonus_from_last_draft_position", "sampling.py",
+     "emission_scores(None, q[b, K], seed, b, K)", "emission_scores(None, q[b, K - 1], seed, b, K)", 1),
     ("softmax_temperature_multiplies", "sampling.py",
      "np.float64) / float(temperature)", "np.float64) * float(temperature)", 1),
     ("accept_and_resample_share_a_stream", "sampling.py", "STREAM_ACCEPT = 2", "STREAM_ACCEPT = 1", 1),
@@ -111,7 +114,8 @@ MUTATIONS = [
 # Runs the statistical pins (seconds each) after the rest, so that most planted
 # slips stop the copy's suite early; the order changes no outcome.
 _ORDER_PLUGIN = """
-SLOW = ("exact_law", "follows_the_target_law", "residual_draw", "acceptance_length_law", "acceptance_rate")
+SLOW = ("exact_law", "follows_the_target_law", "residual_draw", "acceptance_length_law", "acceptance_rate",
+        "draws_from_the_target")
 
 
 def pytest_collection_modifyitems(items):

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 from scipy import special, stats
 
-from oracle import accept_uniform, resample_noise, softmax_rows, verify_sample
+from oracle import accept_uniform, emission_scores, resample_noise, softmax_rows, verify_sample
 
 
 def _first_emitted(res, draft):
@@ -141,3 +141,38 @@ def test_residual_draw_follows_the_normalised_residual():
     assert counts[1] == 0                             # the rejected token has no residual mass
     keep = resid > 0
     assert stats.chisquare(counts[keep], resid[keep] * len(tokens)).pvalue > 1e-3, (counts / len(tokens), resid)
+
+
+def test_empty_residual_draws_from_the_target():
+    # p and q agree in fp64 except at the drafted token, whose probability (~1e-20) is
+    # below fp64 resolution: the acceptance ratio is e^-1, yet max(0, q - p) is zero
+    # everywhere.  The emitted token after such a rejection is drawn from q.
+    T = 1.0
+    dl = np.array([[[0.0, 1.0, 2.0, 0.5, -45.0]]])
+    tl = np.concatenate([dl, [[[0.3, 0.1, 0.2, 0.4, 0.0]]]], axis=1)
+    tl[0, 0, 4] = -46.0
+    p, q = softmax_rows(dl, T)[0, 0], softmax_rows(tl, T)[0, 0]
+    assert not (np.maximum(q - p, 0.0) > 0).any()
+    np.testing.assert_allclose(q[4] / p[4], np.exp(-1.0), rtol=1e-12)
+    draft = np.array([[4]])
+    tokens = []
+    for s in range(6000):
+        res = verify_sample(dl, tl, draft, T, seed=s)
+        if res.tau[0] == 0:
+            tokens.append(int(res.token[0]))
+            assert res.token[0] == np.argmax(np.log(q) + resample_noise(s, 0, 0, 5))
+    assert abs(len(tokens) / 6000 - (1 - np.exp(-1.0))) < 0.03
+    counts = np.bincount(tokens, minlength=5)
+    keep = q > 1e-6
+    assert counts[~keep].sum() == 0
+    assert stats.chisquare(counts[keep], q[keep] / q[keep].sum() * len(tokens)).pvalue > 1e-3, (counts, q)
+
+
+def test_emission_scores_cases():
+    q = np.array([0.1, 0.2, 0.3, 0.4])
+    p = np.array([0.4, 0.1, 0.3, 0.2])
+    g = resample_noise(3, 1, 2, 4)
+    with np.errstate(divide="ignore"):
+        np.testing.assert_array_equal(emission_scores(p, q, 3, 1, 2), np.log([0.0, 0.1, 0.0, 0.2]) + g)
+        np.testing.assert_array_equal(emission_scores(None, q, 3, 1, 2), np.log(q) + g)
+        np.testing.assert_array_equal(emission_scores(q, q, 3, 1, 2), np.log(q) + g)   # empty residual
