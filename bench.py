@@ -315,8 +315,7 @@ def run_ours(args):
 
     import draft_model_b200 as dm
     import synth
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from _harness import device_weights, to_dev, workspace_for
+    from draft_model_b200.tensors import device_weights, to_dev, workspace_for
 
     dm.load_library()
     B = args.batch
@@ -325,7 +324,7 @@ def run_ours(args):
     dw = device_weights(w, dev)
     if args.gate_table:
         # variant: token -> gate table built once per weight set (not timed)
-        from _harness import aligned_workspace
+        from draft_model_b200.tensors import aligned_workspace
         table = torch.empty((cfg.V, 3 * cfg.H), dtype=torch.float32, device=dev)
         dm.domino_build_gate_table(dw, table, workspace=aligned_workspace(1024))
         dw.set_gate_table(table)
@@ -484,8 +483,7 @@ def run_loss(args):
 
     import draft_model_b200 as dm
     import synth
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from _harness import aligned_workspace, device_weights, to_dev
+    from draft_model_b200.tensors import aligned_workspace, device_weights, to_dev
 
     dm.load_library()
     B = args.batch
@@ -558,8 +556,7 @@ def run_verify(args):
     import torch
 
     import draft_model_b200 as dm
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from _harness import aligned_workspace
+    from draft_model_b200.tensors import aligned_workspace
 
     dm.load_library()
     B = args.batch

@@ -19,48 +19,10 @@ import torch
 import draft_model_b200 as dm
 import oracle
 import synth
+from draft_model_b200.tensors import aligned_workspace, device_weights, to_dev, workspace_for  # noqa: F401
 
 MARGIN = 0.05
 TOL = {"bf16": 2e-2, "f32": 1e-4}
-
-
-def to_dev(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
-    """Storage-form numpy array -> contiguous device tensor."""
-    if dtype == "bf16":
-        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
-    elif dtype == "f32":
-        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
-    else:
-        t = torch.from_numpy(np.ascontiguousarray(a))
-    return t.to(device)
-
-
-def device_weights(w: synth.Weights, device="cuda") -> dm.DominoWeights:
-    dt = w.dtype
-    w_lm = to_dev(w.w_lm, dt, device)
-    embed = w_lm if w.embed is w.w_lm else to_dev(w.embed, dt, device)
-    b_ih = None if w.b_ih is None else torch.from_numpy(w.b_ih).to(device)
-    b_hh = None if w.b_hh is None else torch.from_numpy(w.b_hh).to(device)
-    return dm.DominoWeights(w_lm, embed, to_dev(w.w_ih, dt, device), to_dev(w.w_hh, dt, device), b_ih, b_hh,
-                            to_dev(w.w1, dt, device), to_dev(w.w2, dt, device))
-
-
-def aligned_workspace(n: int) -> torch.Tensor:
-    """n bytes of 256-byte aligned device memory with a zeroed control block."""
-    ws = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
-    off = (-ws.data_ptr()) % 256
-    ws = ws[off:off + n]
-    dm.domino_workspace_init(ws)
-    return ws
-
-
-def workspace_for(dw: dm.DominoWeights, B: int, K: int, host: bool = False) -> torch.Tensor:
-    n = dm.domino_workspace_bytes_host(dw, B, K) if host else dm.domino_workspace_bytes(dw, B, K)
-    ws = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
-    off = (-ws.data_ptr()) % 256
-    ws = ws[off:off + n]
-    dm.domino_workspace_init(ws)
-    return ws
 
 
 def run_gpu(dw, cfg: synth.Config, hidden: np.ndarray, anchor: np.ndarray, *, forced=None, target=None,

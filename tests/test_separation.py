@@ -44,6 +44,27 @@ def test_cuda_sources_do_not_reach_into_the_oracle():
             assert "oracle" not in text.lower(), f
 
 
+def test_bench_reaches_the_oracle_only_in_its_cpu_legs():
+    """bench.py imports the oracle only inside the CPU-baseline and reference
+    helpers, and nothing from tests/ (whose harness imports the oracle)."""
+    path = os.path.join(ROOT, "bench.py")
+    tree = ast.parse(open(path).read(), filename=path)
+    allowed = {"oracle_block_rate", "OracleFraction"}
+    for node in tree.body:
+        name = getattr(node, "name", None)
+        sub = ast.Module(body=[node], type_ignores=[])
+        found = set()
+        for n in ast.walk(sub):
+            if isinstance(n, ast.Import):
+                found.update(a.name.split(".")[0] for a in n.names)
+            elif isinstance(n, ast.ImportFrom) and n.module:
+                found.add(n.module.split(".")[0])
+        assert "_harness" not in found, name
+        if "oracle" in found:
+            assert name in allowed, f"bench.py imports the oracle in {name!r}"
+    assert "\"tests\"" not in open(path).read()
+
+
 def test_missing_library_raises(monkeypatch):
     from draft_model_b200 import _binding
     monkeypatch.setattr(_binding, "_lib", None)
