@@ -83,9 +83,26 @@ def load_library() -> ctypes.CDLL:
 # ---------------------------------------------------------------- marshalling helpers
 
 def _ptr(t) -> int | None:
+    """Device pointer: a contiguous CUDA tensor, None, or a raw integer address."""
     if t is None:
         return None
     if isinstance(t, torch.Tensor):
+        if not t.is_cuda:
+            raise ValueError("expected a CUDA tensor (device memory), got a tensor on " + str(t.device))
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        return t.data_ptr()
+    return int(t)
+
+
+def _hptr(t) -> int | None:
+    """Host pointer: a contiguous CPU tensor (pinned memory makes the copies asynchronous),
+    None, or a raw integer address."""
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if t.is_cuda:
+            raise ValueError("expected a host (CPU) tensor, got a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
         return t.data_ptr()
@@ -279,9 +296,9 @@ def domino_draft_block_host(w: DominoWeights, hidden_host, anchor_host, *, mode=
     """Host-buffer variant: host tensors in and out (pinned memory recommended)."""
     B, K = draft_out_host.shape
     wp, wn = _ws(workspace)
-    _check(load_library().domino_draft_block_host(w.ref, _ptr(hidden_host), _ptr(anchor_host), B, K, mode,
-                                                  temperature, seed, _ptr(forced_host), _ptr(target_host),
-                                                  _ptr(draft_out_host), _ptr(tau_out_host), wp, wn,
+    _check(load_library().domino_draft_block_host(w.ref, _hptr(hidden_host), _hptr(anchor_host), B, K, mode,
+                                                  temperature, seed, _hptr(forced_host), _hptr(target_host),
+                                                  _hptr(draft_out_host), _hptr(tau_out_host), wp, wn,
                                                   _stream(stream)), "domino_draft_block_host")
 
 

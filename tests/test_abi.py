@@ -192,3 +192,20 @@ def test_stage_entry_points_validate_on_the_host(lib):
     assert noalloc(B=9) == UNSUP
     assert noalloc(ww=_cw(H=8192)) == UNSUP
     assert noalloc(K=0) == INVALID
+
+
+def test_binding_rejects_host_tensors_for_device_arguments():
+    """A CPU tensor where the C ABI takes device memory raises in the binding,
+    before any call into the library (a host pointer must never reach a kernel)."""
+    import torch
+    from draft_model_b200 import _binding
+    d = torch.zeros((2, 4), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dm.domino_verify(d, d, torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dm.domino_workspace_init(torch.zeros(1024, dtype=torch.uint8))
+    # host-buffer arguments take CPU tensors, raw addresses pass through unchanged
+    assert _binding._hptr(d) == d.data_ptr()
+    assert _binding._ptr(None) is None and _binding._ptr(4096) == 4096
+    with pytest.raises(ValueError, match="contiguous"):
+        _binding._hptr(torch.zeros((4, 4), dtype=torch.int32).t())
