@@ -51,10 +51,14 @@ def dist_env():
 
 
 def init_dist(world: int, backend: str):
+    """Join the process group.  Its timeout (DOMINO_PG_TIMEOUT_S, default 300 s)
+    bounds every collective: when a rank dies, the others' next barrier or
+    all-reduce ends with an error instead of waiting for good."""
     import torch.distributed as dist
     if world > 1 and not dist.is_initialized():
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+        timeout = float(os.environ.get("DOMINO_PG_TIMEOUT_S", "300"))
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout))
 
 
 def barrier(world: int):

@@ -49,6 +49,39 @@ def test_replica_aggregation_max_over_ranks(world):
         assert mx == world - 1
 
 
+def _worker_one_dies(rank, world, port, out):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port), DOMINO_PG_TIMEOUT_S="10")
+    bench.init_dist(world, "gloo")
+    bench.barrier(world)                      # step boundary both ranks reach
+    if rank == world - 1:
+        out[rank] = "left"
+        os._exit(3)                           # this rank dies between steps
+    try:
+        bench.max_over_ranks(1.0, world)      # the survivor's next collective
+        out[rank] = "returned"
+    except Exception as e:                    # noqa: BLE001 - any error ends the wait
+        out[rank] = "raised " + type(e).__name__
+
+
+def test_a_dead_rank_ends_the_others_collective_with_an_error():
+    """Failure detection on the host: a replica that dies between steps makes
+    the surviving rank's next collective fail within the process-group timeout."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_one_dies, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode is not None for p in procs), "a rank is still waiting"
+    assert procs[1].exitcode == 3 and out[1] == "left"
+    assert out[0].startswith("raised"), out[0]
+
+
 def test_single_rank_aggregation():
     value, t = bench.aggregate([0.5, 0.5], 4, 1)
     assert t == 1.0 and value == 8.0
