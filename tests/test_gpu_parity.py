@@ -108,6 +108,24 @@ def test_tiny_f32_config():
 
 @cuda
 @pytest.mark.parametrize("cfg", [
+    small(B=1, K=16, mode="gumbel", temperature=1.0, seed=4),
+    small(B=9, K=7, seed=5),
+    small(B=5, K=6, dtype="f32", seed=9),
+], ids=["persistent_gumbel_b1", "tensor_core_b9", "f32_b5"])
+def test_repeated_blocks_are_bit_identical(cfg):
+    """No float atomics and fixed reduction orders: two runs of the same block give
+    the same picks and bit-identical final logits (a barrier race would not)."""
+    w, m, dw = setup(cfg)
+    hidden, anchor = synth.make_hidden(cfg), synth.make_anchor(cfg)
+    first = run_gpu(dw, cfg, hidden, anchor)
+    second = run_gpu(dw, cfg, hidden, anchor)
+    assert first["status"] == 0 and second["status"] == 0
+    np.testing.assert_array_equal(first["tokens"], second["tokens"])
+    np.testing.assert_array_equal(first["logits"].view(np.uint32), second["logits"].view(np.uint32))
+
+
+@cuda
+@pytest.mark.parametrize("cfg", [
     small(),
     small(B=1, K=16, mode="gumbel", temperature=1.0, seed=4),
     small(B=9, K=7, mode="gumbel", temperature=0.7, seed=5),
