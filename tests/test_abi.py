@@ -4,6 +4,8 @@ arguments synchronously (before any CUDA call)."""
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -209,3 +211,34 @@ def test_binding_rejects_host_tensors_for_device_arguments():
     assert _binding._ptr(None) is None and _binding._ptr(4096) == 4096
     with pytest.raises(ValueError, match="contiguous"):
         _binding._hptr(torch.zeros((4, 4), dtype=torch.int32).t())
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "domino.h"
+int main(void) {
+  domino_weights w;
+  memset(&w, 0, sizeof w);
+  if (strcmp(domino_status_str(DOMINO_ERR_INVALID_ARG), "DOMINO_ERR_INVALID_ARG") != 0) return 1;
+  if (domino_launches_per_block(&w, 1, 16) != -1) return 2;         /* no weights: rejected */
+  if (domino_workspace_bytes(&w, 1, 16) != 0) return 3;
+  if (domino_verify(NULL, NULL, 1, 16, NULL, NULL) != DOMINO_ERR_INVALID_ARG) return 4;
+  puts("ok");
+  return 0;
+}
+"""
+
+
+@pytest.mark.skipif(not shutil.which("gcc"), reason="needs gcc")
+def test_plain_c99_client_compiles_links_and_calls_the_library(lib, tmp_path):
+    """The boundary is a C ABI: a strict C99 program includes the header, links
+    libdomino.so and calls host-side entry points (no GPU needed for these)."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    libdir = os.path.dirname(dm.library_path())
+    exe = tmp_path / "client"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                    str(src), "-L", libdir, "-ldomino", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
