@@ -41,6 +41,12 @@ MUTATIONS = [
     ("sigmoid_sign", "domino_ref.py", "1.0 / (1.0 + np.exp(-x))", "1.0 / (1.0 + np.exp(x))", 1),
     ("silu_is_sigmoid", "domino_ref.py", "return x * sigmoid(x)", "return sigmoid(x)", 1),
     ("widen_bf16_shift", "domino_ref.py", "<< np.uint32(16)", "<< np.uint32(15)", 1),
+    ("gru_biases_dropped", "domino_ref.py",
+     "return np.zeros(H3) if a is None else np.asarray(a, np.float32).astype(np.float64)",
+     "return np.zeros(H3)", 1),
+    ("embedding_read_from_lm_head", "domino_ref.py",
+     "widen_f64(self.embed[np.asarray(tokens, dtype=np.int64)], self.dtype)",
+     "widen_f64(self.w_lm[np.asarray(tokens, dtype=np.int64)], self.dtype)", 1),
     # the correction loop
     ("concat_state_first", "domino_ref.py",
      "np.concatenate([hidden64[:, p, :], s], axis=1)", "np.concatenate([s, hidden64[:, p, :]], axis=1)", 1),
@@ -88,6 +94,9 @@ MUTATIONS = [
      "lse = m + np.log(np.exp(x - m[..., None]).sum(axis=-1))", "lse = np.log(np.exp(x - m[..., None]).sum(axis=-1))", 1),
     ("weights_start_at_gamma", "training.py",
      "np.arange(K, dtype=np.float64)", "np.arange(1, K + 1, dtype=np.float64)", 1),
+    ("base_loss_on_final_logits", "training.py",
+     "ce_base = cross_entropy_rows(base_logits, labels)", "ce_base = cross_entropy_rows(final_logits, labels)", 1),
+    ("weights_normalised_by_k", "training.py", "/ (B * w.sum()))", "/ (B * K))", 2),
     ("mix_swapped", "training.py",
      "(1.0 - lam) * l_final + lam * l_base", "lam * l_final + (1.0 - lam) * l_base", 1),
     ("batch_mean_dropped", "training.py", "/ (B * w.sum()))", "/ w.sum())", 2),
@@ -103,6 +112,8 @@ MUTATIONS = [
     ("empty_residual_fallback_dropped", "sampling.py", "if (resid > 0.0).any():", "if True:", 1),
     ("bonus_from_last_draft_position", "sampling.py",
      "emission_scores(None, q[b, K], seed, b, K)", "emission_scores(None, q[b, K - 1], seed, b, K)", 1),
+    ("no_stop_at_first_rejection", "sampling.py",
+     "                pos = i\n                break", "                pos = i", 1),
     ("softmax_temperature_multiplies", "sampling.py",
      "np.float64) / float(temperature)", "np.float64) * float(temperature)", 1),
     ("accept_and_resample_share_a_stream", "sampling.py", "STREAM_ACCEPT = 2", "STREAM_ACCEPT = 1", 1),
