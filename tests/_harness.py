@@ -78,3 +78,46 @@ def check_against_oracle(model: oracle.Model, cfg: synth.Config, hidden, anchor,
         want = oracle.verify(g_tok, np.asarray(target)[rows])
         np.testing.assert_array_equal(gpu["tau"][rows], want)
     return ref, stats
+
+
+# ---------------------------------------------------------------- stochastic verification
+
+ACCEPT_TIE = 1e-5
+SCORE_TIE = 1e-3
+
+
+def emission_scores_of(dl, tl, b, pos, T, seed):
+    """The oracle's Gumbel-max scores of request b's emitted token after pos accepted drafts."""
+    K = dl.shape[1]
+    q = oracle.softmax_rows(tl[b, pos].astype(np.float64), T)
+    p = oracle.softmax_rows(dl[b, pos].astype(np.float64), T) if pos < K else None
+    return oracle.emission_scores(p, q, seed, b, pos)
+
+
+def check_verify_sample(dl, tl, draft, T, seed, tau, tok):
+    """Comparison protocol of stochastic verification.
+
+    Floating point decides integers here (accept or reject; the Gumbel-max
+    draw).  A request whose acceptance test at any examined position lies within
+    ACCEPT_TIE of its threshold (|u - min(1, q/p)|) is a precision tie and only
+    checked for validity.  Otherwise tau must match the oracle exactly, and the
+    emitted token must score within SCORE_TIE of the oracle's best draw (it is
+    the oracle's own pick wherever the oracle's top-2 margin exceeds that).
+    """
+    ref = oracle.verify_sample(dl.astype(np.float64), tl.astype(np.float64), draft, T, seed)
+    B, K, V = dl.shape
+    stats = {"compared": 0, "ties": 0, "rejected": 0}
+    for b in range(B):
+        assert 0 <= tau[b] <= K and 0 <= tok[b] < V
+        examined = min(int(ref.tau[b]) + 1, K)
+        margin = np.abs(ref.uniform[b, :examined] - np.minimum(1.0, ref.ratio[b, :examined]))
+        if (margin < ACCEPT_TIE).any():
+            stats["ties"] += 1
+            continue
+        assert tau[b] == ref.tau[b], (b, tau[b], ref.tau[b])
+        score = emission_scores_of(dl, tl, b, int(ref.tau[b]), T, seed)
+        assert np.isfinite(score[tok[b]]), (b, tok[b])
+        assert score[tok[b]] >= score.max() - SCORE_TIE, (b, tok[b], int(np.argmax(score)))
+        stats["compared"] += 1
+        stats["rejected"] += int(ref.tau[b] < K)
+    return stats

@@ -6,14 +6,16 @@ it gets outputs made on the CPU, in the form the device path returns them
 same block with one planted error must fail. The planted errors are a pick
 changed where the oracle's margin exceeds 0.05, one logit moved past the
 tolerance, a tau off by one, and a teacher-forced pick that is not the best.
-Small deviations inside the stated tolerances must still pass.
+Small deviations inside the stated tolerances must still pass.  The same holds
+for the stochastic-verification protocol: a tau off by one, a poor or
+out-of-range emitted token fail it.
 """
 import numpy as np
 import pytest
 
 import oracle
 import synth
-from _harness import MARGIN, TOL, check_against_oracle
+from _harness import MARGIN, SCORE_TIE, TOL, check_against_oracle, check_verify_sample, emission_scores_of
 
 
 def _setup(dtype, mode):
@@ -84,3 +86,41 @@ def test_teacher_forced_pick_that_is_not_the_best_fails():
     bad["tokens"][b, p] = (bad["tokens"][b, p] + 1) % cfg.V
     with pytest.raises(AssertionError, match="picks off"):
         check_against_oracle(model, cfg, hidden, anchor, bad, forced=forced)
+
+
+# ---------------------------------------------------------------- stochastic verification
+
+def _verify_case():
+    rng = np.random.default_rng(31)
+    B, K, V = 12, 4, 200
+    dl = rng.normal(0.0, 2.0, size=(B, K, V)).astype(np.float32)
+    tl = np.concatenate([dl + rng.normal(0.0, 0.8, size=(B, K, V)), rng.normal(0.0, 2.0, size=(B, 1, V))],
+                        axis=1).astype(np.float32)
+    draft = rng.integers(0, V, size=(B, K)).astype(np.int32)
+    ref = oracle.verify_sample(dl.astype(np.float64), tl.astype(np.float64), draft, 1.0, 17)
+    return dl, tl, draft, ref
+
+
+def test_verify_gate_passes_the_oracles_own_result():
+    dl, tl, draft, ref = _verify_case()
+    stats = check_verify_sample(dl, tl, draft, 1.0, 17, ref.tau, ref.token)
+    assert stats["compared"] + stats["ties"] == len(ref.tau) and stats["compared"] >= len(ref.tau) - 1
+
+
+def test_verify_gate_rejects_a_wrong_tau_or_token():
+    dl, tl, draft, ref = _verify_case()
+    K, V = dl.shape[1], dl.shape[2]
+    b = int(np.flatnonzero(ref.tau < K)[0])
+    tau = ref.tau.copy()
+    tau[b] += 1
+    with pytest.raises(AssertionError):
+        check_verify_sample(dl, tl, draft, 1.0, 17, tau, ref.token)
+    score = emission_scores_of(dl, tl, b, int(ref.tau[b]), 1.0, 17)
+    tok = ref.token.copy()
+    tok[b] = int(np.argmin(np.where(np.isfinite(score), score, np.inf)))   # a valid but poor draw
+    assert score[tok[b]] < score.max() - SCORE_TIE
+    with pytest.raises(AssertionError):
+        check_verify_sample(dl, tl, draft, 1.0, 17, ref.tau, tok)
+    tok[b] = V                                                           # out of range
+    with pytest.raises(AssertionError):
+        check_verify_sample(dl, tl, draft, 1.0, 17, ref.tau, tok)
